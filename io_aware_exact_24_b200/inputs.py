@@ -1,0 +1,124 @@
+"""Seeded synthetic inputs for the attention forward (shared by tests, bench, oracle checks).
+
+This module only draws numbers and rounds them to bf16; it contains none of
+the attention arithmetic, so both the CUDA path and the CPU oracle can consume
+its output without sharing any of the method's code.
+
+Recipe (stated once, used everywhere):
+
+* generator: numpy's ``Philox`` bit generator (Philox4x64-10, Salmon et al.,
+  "Parallel random numbers: as easy as 1, 2, 3", SC'11), one independent stream
+  per tensor, keyed by ``seed * 16 + tensor_id`` with tensor_id Q=0, K=1, V=2,
+  key_lens=3;
+* values: ``standard_normal`` in float32 times sigma (sigma = 1 or 0.5, both
+  exact in float32), rounded to bf16 with round-to-nearest-even;
+* key lengths: integers uniform on [lo, hi] inclusive, one per sequence,
+  shared by all heads.
+
+The workload shapes stand in for the pages' benchmarks (GPT-2 at 1K, a
+BERT-large encoder with padding, Long-Range-Arena-like long sequences); their
+datasets and weights are not used -- only the shapes, mask kinds and value
+distributions.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_KEYLEN = 0, 1, 2, 3
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention-forward problem: shapes, mask kind, value distribution, seed."""
+
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    scale: float
+    sigma: float = 1.0
+    key_len_range: tuple[int, int] | None = None  # inclusive; None = no padding
+    seed: int = 0
+
+    @property
+    def flop(self) -> float:
+        """4*B*H*Nq*Nk*d, causal counted as exactly half."""
+        f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
+        return f / 2.0 if self.causal else f
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """Every operand moved once: Q,K,V read and O written as bf16, LSE as fp32."""
+        return (2 * self.B * self.H * self.d * (2 * self.Nq + 2 * self.Nk)
+                + 4 * self.B * self.H * self.Nq)
+
+    def describe(self) -> str:
+        mask = "causal" if self.causal else "none"
+        if self.key_len_range:
+            mask = f"key_len~U{{{self.key_len_range[0]}..{self.key_len_range[1]}}}"
+        return (f"B{self.B} H{self.H} Nq{self.Nq} Nk{self.Nk} d{self.d} mask={mask} "
+                f"sigma={self.sigma} scale={self.scale:.6g} seed={self.seed}")
+
+
+# The five problems the library is measured and checked on.
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 128, 128, 64, False, 1 / 8, 1.0, None, 1),
+    "gpt2_causal_1k": Workload("gpt2_causal_1k", 8, 12, 1024, 1024, 64, True, 1 / 8,
+                               1.0, None, 2),
+    "bert_padded_512": Workload("bert_padded_512", 16, 16, 512, 512, 64, False, 1 / 8,
+                                1.0, (128, 512), 3),
+    "long_16k_d64": Workload("long_16k_d64", 1, 16, 16384, 16384, 64, False, 1 / 8,
+                             1.0, None, 4),
+    "causal_8000_d128": Workload("causal_8000_d128", 2, 32, 8000, 8000, 128, True,
+                                 float(np.float32(1 / math.sqrt(128))), 0.5, None, 5),
+}
+WORKLOAD_ORDER = ["tiny", "gpt2_causal_1k", "bert_padded_512", "long_16k_d64",
+                  "causal_8000_d128"]
+
+
+def _rng(seed: int, tensor_id: int) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(key=int(seed) * 16 + int(tensor_id)))
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round-to-nearest-even); returns uint16 bit patterns."""
+    x = np.asarray(x, dtype=np.float32)
+    u = np.ascontiguousarray(x).reshape(-1).view(np.uint32).astype(np.uint64)
+    rounded = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return rounded.astype(np.uint16).reshape(x.shape)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).reshape(b.shape)
+
+
+def normal_bf16(shape, seed: int, tensor_id: int, sigma: float = 1.0) -> np.ndarray:
+    """N(0, sigma^2) samples rounded to bf16, as uint16 bit patterns."""
+    x = _rng(seed, tensor_id).standard_normal(size=shape, dtype=np.float32)
+    if sigma != 1.0:
+        x *= np.float32(sigma)
+    return f32_to_bf16_bits(x)
+
+
+def key_lengths(B: int, lo: int, hi: int, seed: int) -> np.ndarray:
+    """Per-sequence key lengths, uniform on the integers [lo, hi]."""
+    return _rng(seed, TENSOR_KEYLEN).integers(lo, hi + 1, size=B, dtype=np.int64).astype(np.int32)
+
+
+def make_inputs(w: Workload):
+    """Return dict(q, k, v: uint16 bf16 bits [B,H,N,d]; key_lens: int32 [B] or None)."""
+    q = normal_bf16((w.B, w.H, w.Nq, w.d), w.seed, TENSOR_Q, w.sigma)
+    k = normal_bf16((w.B, w.H, w.Nk, w.d), w.seed, TENSOR_K, w.sigma)
+    v = normal_bf16((w.B, w.H, w.Nk, w.d), w.seed, TENSOR_V, w.sigma)
+    kl = None
+    if w.key_len_range is not None:
+        kl = key_lengths(w.B, w.key_len_range[0], w.key_len_range[1], w.seed)
+    return {"q": q, "k": k, "v": v, "key_lens": kl}

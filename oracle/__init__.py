@@ -1,0 +1,142 @@
+"""fp64 CPU oracle for the exact attention forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg (and its ``--impl reference`` arm) may import this package.  The product
+path (``io_aware_exact_24_b200``) never does, and this package never imports
+the product.
+
+Two independent C formulations are wrapped here:
+
+* ``attn_ref``    (attn_ref.c): the plain definition, S and P materialised per
+  row -- "FlashAttention 与边缘设备上的注意力内存瓶颈", section 2, and
+  "FlashAttention：把注意力从公式写成数据流", opening paragraph.
+* ``attn_online`` (attn_online.c): the block-wise online-softmax recurrence --
+  "FlashAttention：把注意力从公式写成数据流", section "分块与在线 softmax".
+
+Inputs are bf16 *bit patterns* (``numpy.uint16``) so that the oracle sees
+exactly the bytes the GPU sees; outputs are fp64 and never rounded.
+
+Pins (what ties this oracle to something other than itself) live in
+``tests/test_oracle_pins.py`` and ``tests/test_golden.py``.  The GPU-internal
+rounding of P to bf16 has no counterpart here: "parity unpinned" for that
+detail, bounded only by the stated output tolerances.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SOURCES = ("attn_ref.c", "attn_online.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, OpenMP)."""
+    srcs = [os.path.join(_HERE, s) for s in _SOURCES]
+    if not force and os.path.exists(_LIB_PATH):
+        lib_mtime = os.path.getmtime(_LIB_PATH)
+        if all(os.path.getmtime(s) <= lib_mtime for s in srcs):
+            return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-Wall",
+           "-o", tmp, *srcs, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            vp = ctypes.c_void_p
+            lib.attn_ref_fp64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                          f32, i32, vp, vp, vp]
+            lib.attn_ref_fp64.restype = i32
+            lib.attn_ref_fp64_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
+                                               i64, f32, i32, vp, i64, vp, vp]
+            lib.attn_ref_fp64_rows.restype = i32
+            lib.attn_online_fp64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
+                                             i64, f32, i32, i64, vp, vp]
+            lib.attn_online_fp64.restype = i32
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = i32
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (set OMP_NUM_THREADS to change)."""
+    return int(_load().oracle_num_threads())
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(q, k, v, key_lens):
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be [B,H,N,d] bf16 bit arrays")
+    B, H, Nq, d = q.shape
+    if k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("shape mismatch between q, k, v")
+    if key_lens is not None:
+        key_lens = np.ascontiguousarray(key_lens, dtype=np.int32)
+        if key_lens.shape != (B,):
+            raise ValueError("key_lens must be int32 [B]")
+    return q, k, v, key_lens, B, H, Nq, k.shape[2], d
+
+
+def attn_ref(q, k, v, scale, causal=False, key_lens=None, return_p=False):
+    """Plain definition.  Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq][, P])."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    o = np.empty((B, H, Nq, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    p = np.empty((B, H, Nq, Nk), np.float64) if return_p else None
+    rc = _load().attn_ref_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
+                               Nq, Nk, d, float(np.float32(scale)), int(bool(causal)),
+                               _ptr(o), _ptr(lse), _ptr(p))
+    if rc != 0:
+        raise RuntimeError(f"attn_ref_fp64 failed ({rc})")
+    return (o, lse, p) if return_p else (o, lse)
+
+
+def attn_ref_rows(q, k, v, scale, row_ids, causal=False, key_lens=None):
+    """Definition on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n])."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    rows = np.ascontiguousarray(row_ids, dtype=np.int64)
+    o = np.empty((rows.size, d), np.float64)
+    lse = np.empty((rows.size,), np.float64)
+    rc = _load().attn_ref_fp64_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
+                                    Nq, Nk, d, float(np.float32(scale)),
+                                    int(bool(causal)), _ptr(rows), rows.size,
+                                    _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise RuntimeError(f"attn_ref_fp64_rows failed ({rc})")
+    return o, lse
+
+
+def attn_online(q, k, v, scale, causal=False, key_lens=None, block=7):
+    """Online-softmax formulation.  Returns (O fp64, LSE fp64)."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    o = np.empty((B, H, Nq, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    rc = _load().attn_online_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
+                                  Nq, Nk, d, float(np.float32(scale)),
+                                  int(bool(causal)), int(block), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise RuntimeError(f"attn_online_fp64 failed ({rc})")
+    return o, lse

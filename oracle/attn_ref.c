@@ -1,0 +1,193 @@
+/*
+ * oracle/attn_ref.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, fp64 CPU oracle for the exact attention forward pass
+ *     O = softmax(scale * Q K^T + mask) V,   LSE_i = ln sum_j exp(scale * q_i . k_j)
+ * written straight from the definition: for every query row the full score
+ * row S_i and probability row P_i are materialised, then O_i = P_i V.
+ *
+ * Sources for what is computed:
+ *   - "FlashAttention 与边缘设备上的注意力内存瓶颈", section 2 (standard
+ *     attention forms S and P, both N x N) and section 3.2 (the tiled method
+ *     stays exact, so its result is this definition).
+ *   - "FlashAttention：把注意力从公式写成数据流", opening paragraph (S = QK^T,
+ *     then softmax, then multiply by V) and section "精度、掩码和边界情况"
+ *     (masked positions never enter the normaliser; tail blocks).
+ * Readings where the pages are silent (causal alignment, key_lens, LSE,
+ * fully masked rows) are the ones the library documents in include/fa.h:
+ *   - causal is bottom-right aligned: key j is visible to query i iff
+ *     j <= i + (N_k - N_q);
+ *   - key_lens[b] (NULL = all keys) is clamped to [0, N_k]; keys j >= it are masked;
+ *   - both masks combine with AND; the valid keys of row i are therefore the
+ *     prefix [0, lim_i);
+ *   - a row with no valid key has O = 0 and LSE = -inf.
+ *
+ * Nothing here is shared with the CUDA path.  Only tests/, the package's
+ * graft entry smoke check and bench.py's CPU baseline may call it.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 bit pattern -> fp64, exact (bf16 is the top half of an fp32). */
+static double bf16_bits_to_f64(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Number of valid keys of query row i: the prefix [0, lim) of the key axis. */
+static int64_t row_limit(int64_t i, int64_t b, const int32_t *key_lens,
+                         int64_t Nq, int64_t Nk, int causal) {
+    int64_t kl = Nk;
+    if (key_lens) {
+        kl = key_lens[b];
+        if (kl < 0) kl = 0;
+        if (kl > Nk) kl = Nk;
+    }
+    int64_t lim = kl;
+    if (causal) {
+        int64_t c = i + (Nk - Nq) + 1; /* keys j <= i + Nk - Nq */
+        if (c < 0) c = 0;
+        if (c < lim) lim = c;
+    }
+    return lim;
+}
+
+/*
+ * One query row, straight from the definition.  s_row and p_row are caller
+ * scratch of length Nk; on return they hold S_i (masked entries -inf) and
+ * P_i (masked entries 0).
+ */
+static void one_row(const uint16_t *q_row, const uint16_t *k_head,
+                    const uint16_t *v_head, int64_t Nk, int64_t d,
+                    double scale, int64_t lim, double *s_row, double *p_row,
+                    double *o_row, double *lse_out) {
+    /* S_ij = scale * sum_c q_ic k_jc for valid j, -inf for masked j. */
+    for (int64_t j = 0; j < Nk; ++j) {
+        if (j < lim) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c)
+                dot += bf16_bits_to_f64(q_row[c]) * bf16_bits_to_f64(k_head[j * d + c]);
+            s_row[j] = scale * dot;
+        } else {
+            s_row[j] = -INFINITY;
+        }
+    }
+    if (lim == 0) {
+        for (int64_t j = 0; j < Nk; ++j) p_row[j] = 0.0;
+        for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    /* softmax over the valid entries: subtract the row max, exp, normalise. */
+    double m = -INFINITY;
+    for (int64_t j = 0; j < lim; ++j)
+        if (s_row[j] > m) m = s_row[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < Nk; ++j) {
+        p_row[j] = (j < lim) ? exp(s_row[j] - m) : 0.0;
+        l += p_row[j];
+    }
+    for (int64_t j = 0; j < Nk; ++j) p_row[j] /= l;
+    /* O_i = sum_j P_ij V_j */
+    for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
+    for (int64_t j = 0; j < lim; ++j)
+        for (int64_t c = 0; c < d; ++c)
+            o_row[c] += p_row[j] * bf16_bits_to_f64(v_head[j * d + c]);
+    *lse_out = m + log(l);
+}
+
+/*
+ * Full forward.  q: bf16 bits [B,H,Nq,d]; k, v: bf16 bits [B,H,Nk,d];
+ * key_lens: int32 [B] or NULL.  o: fp64 [B,H,Nq,d]; lse: fp64 [B,H,Nq].
+ * p_out: NULL, or fp64 [B,H,Nq,Nk] receiving the materialised P.
+ * scale is the fp32 value the GPU receives, widened to fp64.
+ * Returns 0, or -1 on bad sizes / allocation failure.
+ */
+int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                  int64_t Nk, int64_t d, float scale, int causal, double *o,
+                  double *lse, double *p_out) {
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0) return -1;
+    const double sc = (double)scale;
+    const int64_t rows = B * H * Nq;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s_row = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        double *p_row = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        if (!s_row || !p_row) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t r = 0; r < rows; ++r) {
+                const int64_t i = r % Nq;
+                const int64_t bh = r / Nq;
+                const int64_t b = bh / H;
+                const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
+                one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
+                        lim, s_row, p_row, o + r * d, lse + r);
+                if (p_out) memcpy(p_out + r * Nk, p_row, sizeof(double) * (size_t)Nk);
+            }
+        }
+        free(s_row);
+        free(p_row);
+    }
+    return failed ? -1 : 0;
+}
+
+/*
+ * Same definition evaluated only on selected rows, for checking outputs of
+ * problems too large to evaluate whole.  row_ids[n] are flat row indices
+ * r = (b*H + h)*Nq + i.  o_rows: fp64 [n,d]; lse_rows: fp64 [n].
+ */
+int attn_ref_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                       int64_t Nk, int64_t d, float scale, int causal,
+                       const int64_t *row_ids, int64_t n, double *o_rows,
+                       double *lse_rows) {
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0 || n < 0) return -1;
+    const double sc = (double)scale;
+    const int64_t rows = B * H * Nq;
+    for (int64_t t = 0; t < n; ++t)
+        if (row_ids[t] < 0 || row_ids[t] >= rows) return -1;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s_row = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        double *p_row = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        if (!s_row || !p_row) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < n; ++t) {
+                const int64_t r = row_ids[t];
+                const int64_t i = r % Nq;
+                const int64_t bh = r / Nq;
+                const int64_t b = bh / H;
+                const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
+                one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
+                        lim, s_row, p_row, o_rows + t * d, lse_rows + t);
+            }
+        }
+        free(s_row);
+        free(p_row);
+    }
+    return failed ? -1 : 0;
+}

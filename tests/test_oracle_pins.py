@@ -1,0 +1,251 @@
+"""Pins for the fp64 CPU oracle: things the mathematics fixes, checked without the oracle's own code.
+
+Each test below would fail for a plausible slip in the oracle (dropped scale,
+wrong sign, transposed operand, off-by-one in a mask, wrong normaliser):
+
+* rows of the materialised P sum to one (softmax normalisation);
+* the online-softmax formulation agrees with the two-pass one (the pages
+  state the tiled/online result is identical, only the order differs --
+  "FlashAttention：把注意力从公式写成数据流", section "分块与在线 softmax");
+* closed forms: Q = 0 gives the mean of the visible V rows and LSE = ln|J|;
+  a single visible key gives that key's V row and LSE = scale*q.k;
+* invariances: constant V column, key shift, joint K/V permutation, garbage
+  at masked positions, a dominant score;
+* a library routine the special case reduces to: torch's CPU
+  scaled_dot_product_attention in float64 with an explicit boolean mask.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from io_aware_exact_24_b200.inputs import bf16_bits_to_f32, f32_to_bf16_bits, normal_bf16
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _rand(B, H, Nq, Nk, d, seed, sigma=1.0):
+    q = normal_bf16((B, H, Nq, d), seed, 0, sigma)
+    k = normal_bf16((B, H, Nk, d), seed, 1, sigma)
+    v = normal_bf16((B, H, Nk, d), seed, 2, sigma)
+    return q, k, v
+
+
+def _bits(x):
+    """Exactly-representable float values -> bf16 bits (asserts exactness)."""
+    x = np.asarray(x, np.float32)
+    b = f32_to_bf16_bits(x)
+    assert np.array_equal(bf16_bits_to_f32(b), x), "value not exact in bf16"
+    return b
+
+
+def _visible(Nq, Nk, causal, kl):
+    """Boolean [Nq, Nk] visibility written from the documented reading."""
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    vis = np.broadcast_to(j < kl, (Nq, Nk))
+    if causal:
+        vis = vis & (j <= i + (Nk - Nq))
+    return vis
+
+
+CASES = [
+    # B, H, Nq, Nk, d, causal, key_lens
+    (2, 3, 37, 53, 16, False, None),
+    (2, 3, 53, 37, 16, True, None),      # Nq > Nk: leading rows fully masked
+    (2, 2, 41, 41, 8, True, None),
+    (3, 2, 29, 45, 16, False, [0, 17, 45]),
+    (3, 2, 45, 45, 16, True, [5, 45, 60]),  # key_len beyond Nk clamps
+    (1, 1, 1, 1, 4, False, None),
+    (1, 2, 5, 0, 8, False, None),           # no keys at all
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_p_rows_sum_to_one(case):
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 11)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o, lse, p = oracle.attn_ref(q, k, v, 0.25, causal, kl_arr, return_p=True)
+    for b in range(B):
+        klb = Nk if kl is None else min(max(kl[b], 0), Nk)
+        vis = _visible(Nq, Nk, causal, klb)
+        for h in range(H):
+            sums = p[b, h].sum(axis=1)
+            has = vis.any(axis=1)
+            np.testing.assert_allclose(sums[has], 1.0, rtol=0, atol=1e-12)
+            assert np.all(p[b, h][~vis] == 0.0)
+            assert np.all(np.isneginf(lse[b, h][~has]))
+            assert np.all(o[b, h][~has] == 0.0)
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("block", [1, 7, 128])
+def test_online_matches_two_pass(case, block):
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 12)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o1, l1 = oracle.attn_ref(q, k, v, 0.3, causal, kl_arr)
+    o2, l2 = oracle.attn_online(q, k, v, 0.3, causal, kl_arr, block=block)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    fin = np.isfinite(l1)
+    assert np.array_equal(fin, np.isfinite(l2))
+    np.testing.assert_allclose(l2[fin], l1[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_online_matches_two_pass_tiny_workload():
+    from io_aware_exact_24_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS["tiny"]
+    x = make_inputs(w)
+    o1, l1 = oracle.attn_ref(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    o2, l2 = oracle.attn_online(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,kl", [(False, None), (True, None), (False, [7, 30]),
+                                       (True, [3, 30])])
+def test_zero_query_gives_mean_of_visible_values(causal, kl):
+    B, H, Nq, Nk, d = 2, 2, 24, 30, 8
+    _, k, v = _rand(B, H, Nq, Nk, d, 13)
+    q = np.zeros((B, H, Nq, d), np.uint16)          # +0.0 in bf16
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o, lse = oracle.attn_ref(q, k, v, 0.7, causal, kl_arr)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    for b in range(B):
+        vis = _visible(Nq, Nk, causal, Nk if kl is None else kl[b])
+        for h in range(H):
+            for i in range(Nq):
+                n = int(vis[i].sum())
+                if n == 0:
+                    assert np.all(o[b, h, i] == 0) and np.isneginf(lse[b, h, i])
+                    continue
+                np.testing.assert_allclose(o[b, h, i], vf[b, h, vis[i]].mean(axis=0),
+                                           rtol=0, atol=1e-13)
+                assert abs(lse[b, h, i] - math.log(n)) < 1e-13
+
+
+def test_single_key_returns_its_value_row():
+    B, H, Nq, d = 2, 3, 9, 16
+    q, k, v = _rand(B, H, Nq, 1, d, 14)
+    o, lse = oracle.attn_ref(q, k, v, 0.125)
+    qf = bf16_bits_to_f32(q).astype(np.float64)
+    kf = bf16_bits_to_f32(k).astype(np.float64)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    assert np.array_equal(o, np.broadcast_to(vf, o.shape))      # exact: P = 1
+    dots = np.einsum("bhid,bhjd->bhij", qf, kf)[..., 0]
+    np.testing.assert_allclose(lse, 0.125 * dots, rtol=1e-14, atol=1e-14)
+
+
+def test_causal_first_row_sees_only_first_key():
+    B, H, N, d = 1, 4, 33, 16
+    q, k, v = _rand(B, H, N, N, d, 15)
+    o, lse = oracle.attn_ref(q, k, v, 0.125, causal=True)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    assert np.array_equal(o[:, :, 0, :], vf[:, :, 0, :])
+
+
+def test_constant_value_column_is_reproduced():
+    B, H, Nq, Nk, d = 2, 2, 17, 40, 8
+    q, k, v = _rand(B, H, Nq, Nk, d, 16)
+    v = v.copy()
+    v[..., 3] = _bits(1.5)
+    v[..., 5] = _bits(-0.375)
+    for causal, kl in ((False, None), (True, np.array([40, 9], np.int32))):
+        o, _ = oracle.attn_ref(q, k, v, 0.2, causal, kl)
+        np.testing.assert_allclose(o[..., 3], 1.5, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(o[..., 5], -0.375, rtol=0, atol=1e-14)
+
+
+def test_key_shift_leaves_output_and_moves_lse():
+    # small integers: every sum stays exact in bf16 and fp64
+    rng = np.random.default_rng(0)
+    B, H, Nq, Nk, d = 1, 2, 12, 20, 4
+    qv = rng.integers(-2, 3, size=(B, H, Nq, d)).astype(np.float32)
+    kv = rng.integers(-2, 3, size=(B, H, Nk, d)).astype(np.float32)
+    vv = rng.integers(-4, 5, size=(B, H, Nk, d)).astype(np.float32)
+    w = np.array([1, -2, 0, 3], np.float32)
+    scale = 0.25
+    o1, l1 = oracle.attn_ref(_bits(qv), _bits(kv), _bits(vv), scale, causal=True)
+    o2, l2 = oracle.attn_ref(_bits(qv), _bits(kv + w), _bits(vv), scale, causal=True)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-13)
+    shift = scale * (qv.astype(np.float64) @ w.astype(np.float64))
+    np.testing.assert_allclose(l2 - l1, shift, rtol=0, atol=1e-12)
+
+
+def test_joint_key_value_permutation_and_query_permutation():
+    B, H, Nq, Nk, d = 1, 2, 19, 31, 16
+    q, k, v = _rand(B, H, Nq, Nk, d, 17)
+    o1, l1 = oracle.attn_ref(q, k, v, 0.125)
+    perm = np.random.default_rng(1).permutation(Nk)
+    o2, l2 = oracle.attn_ref(q, k[:, :, perm], v[:, :, perm], 0.125)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-13)
+    qperm = np.random.default_rng(2).permutation(Nq)
+    o3, l3 = oracle.attn_ref(q[:, :, qperm], k, v, 0.125)
+    assert np.array_equal(o3, o1[:, :, qperm]) and np.array_equal(l3, l1[:, :, qperm])
+
+
+def test_masked_positions_never_contribute():
+    B, H, Nq, Nk, d = 2, 2, 40, 40, 16
+    q, k, v = _rand(B, H, Nq, Nk, d, 18)
+    kl = np.array([25, 33], np.int32)
+    o1, l1 = oracle.attn_ref(q, k, v, 0.125, True, kl)
+    k2, v2 = k.copy(), v.copy()
+    garbage = _bits(np.float32(8192.0))
+    for b in range(B):
+        k2[b, :, kl[b]:] = garbage
+        v2[b, :, kl[b]:] = _bits(np.float32(-8192.0))
+    o2, l2 = oracle.attn_ref(q, k2, v2, 0.125, True, kl)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    o3, l3 = oracle.attn_online(q, k2, v2, 0.125, True, kl)
+    np.testing.assert_allclose(o3, o1, rtol=0, atol=1e-12)
+
+
+def test_dominant_score_selects_its_value_row():
+    B, H, Nq, Nk, d = 1, 1, 3, 16, 4
+    q = np.zeros((B, H, Nq, d), np.float32)
+    q[..., 0] = 1.0
+    k = np.zeros((B, H, Nk, d), np.float32)
+    k[0, 0, 5, 0] = 100.0                       # score 100 above every other
+    v = np.random.default_rng(3).integers(-3, 4, size=(B, H, Nk, d)).astype(np.float32)
+    o, lse = oracle.attn_ref(_bits(q), _bits(k), _bits(v), 1.0)
+    np.testing.assert_allclose(o[0, 0], np.broadcast_to(v[0, 0, 5], (Nq, d)), rtol=0,
+                               atol=1e-40 + 20 * math.exp(-100) * 4)
+    np.testing.assert_allclose(lse, 100.0 + math.log1p(15 * math.exp(-100)), rtol=0,
+                               atol=1e-13)
+
+
+@pytest.mark.parametrize("case", CASES[:5])
+def test_matches_torch_sdpa_float64(case):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 19)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    scale = 0.2
+    o, lse = oracle.attn_ref(q, k, v, scale, causal, kl_arr)
+    tq, tk, tv = (torch.from_numpy(bf16_bits_to_f32(x).astype(np.float64)) for x in (q, k, v))
+    mask = np.zeros((B, 1, Nq, Nk), bool)
+    for b in range(B):
+        mask[b, 0] = _visible(Nq, Nk, causal, Nk if kl is None else kl[b])
+    tmask = torch.from_numpy(mask)
+    ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=tmask,
+                                         scale=float(np.float32(scale))).numpy()
+    scores = torch.einsum("bhid,bhjd->bhij", tq, tk) * float(np.float32(scale))
+    ref_lse = torch.logsumexp(scores.masked_fill(~tmask, float("-inf")), dim=-1).numpy()
+    has = np.broadcast_to(mask.any(axis=-1), (B, H, Nq))
+    np.testing.assert_allclose(o[has], ref[has], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[has], ref_lse[has], rtol=0, atol=1e-12)
+
+
+def test_rows_entry_matches_full_evaluation():
+    B, H, Nq, Nk, d = 2, 3, 21, 34, 16
+    q, k, v = _rand(B, H, Nq, Nk, d, 20)
+    kl = np.array([34, 11], np.int32)
+    o, lse = oracle.attn_ref(q, k, v, 0.125, True, kl)
+    rows = np.array([0, 5, 20, 21, 63, 64, B * H * Nq - 1], np.int64)
+    orow, lrow = oracle.attn_ref_rows(q, k, v, 0.125, rows, True, kl)
+    assert np.array_equal(orow, o.reshape(-1, d)[rows])
+    assert np.array_equal(lrow, lse.reshape(-1)[rows])
