@@ -1,0 +1,365 @@
+#!/usr/bin/env python3
+"""Throughput of the exact attention forward on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one ``fa_fwd`` call over the whole workload (inputs resident in
+HBM).  Between timed steps the L2 is flushed by writing a 256 MiB buffer
+outside the timed events.  Each step is timed with CUDA events on the
+launching stream; ``ms_per_step`` is the mean, the job time is the max over
+ranks.  Under torchrun every rank runs its own replica of the workload
+(independent problems, no collective on the data path): weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded row
+sample of the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from io_aware_exact_24_b200.inputs import WORKLOADS, WORKLOAD_ORDER, make_inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "causal_8000_d128"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["io_aware_exact_24_b200/csrc/fa_fwd_kernel.cuh",
+                  "io_aware_exact_24_b200/csrc/sm100_ptx.cuh",
+                  "io_aware_exact_24_b200/csrc/fa_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current kernel."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def upload(x, device):
+    import torch
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    kl = None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).to(device)
+    return dev(x["q"]), dev(x["k"]), dev(x["v"]), kl
+
+
+def time_device(w, x, steps, warmup, device, rank, world, clocks=None):
+    """Mean per-launch device time (ms) of fa_fwd on resident inputs, L2 flushed between launches."""
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd
+    q, k, v, kl = upload(x, device)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        fa_fwd(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl, stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s, e in ev:
+        flush.zero_()
+        s.record(stream)
+        launch()
+        e.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    per = [s.elapsed_time(e) for s, e in ev]
+    del q, k, v, o, lse, flush
+    return float(np.mean(per)), per, clk
+
+
+def time_e2e(w, x, steps, warmup, device):
+    """The same forward through the host-buffer C entry point: H2D + kernel + D2H per step."""
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd_host, fa_fwd_host_workspace_size
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    hq, hk, hv = pin(x["q"]), pin(x["k"]), pin(x["v"])
+    hkl = None if x["key_lens"] is None else pin(x["key_lens"])
+    ho = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.int16).pin_memory()
+    hl = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+    ws_bytes = fa_fwd_host_workspace_size(w.B, w.H, w.Nq, w.Nk, w.d, hkl is not None)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fa_fwd_host(hq, hk, hv, ho, hl, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, hkl, ws,
+                    ws_bytes, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + (0 if hkl is None else hkl.numel() * 4)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    del ws
+    return ms, h2d, d2h
+
+
+def oracle_sample_rate(w, x, target_s, rng_seed=0):
+    """Oracle TFLOP/s on a random row sample of the workload sized to ~target_s seconds."""
+    import oracle
+    total_rows = w.B * w.H * w.Nq
+    flop_per_row = w.flop / total_rows
+    rng = np.random.default_rng(rng_seed)
+    n = min(64, total_rows)
+    rows = rng.choice(total_rows, size=n, replace=False)
+    t0 = time.perf_counter()
+    oracle.attn_ref_rows(x["q"], x["k"], x["v"], w.scale, rows, w.causal, x["key_lens"])
+    t = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(total_rows, max(n, n * target_s / t)))
+    rows = rng.choice(total_rows, size=n, replace=False)
+    t0 = time.perf_counter()
+    oracle.attn_ref_rows(x["q"], x["k"], x["v"], w.scale, rows, w.causal, x["key_lens"])
+    t = time.perf_counter() - t0
+    return n * flop_per_row / t / 1e12, n, t, oracle.num_threads()
+
+
+def config_of(w, l2_note, parallelism):
+    mask = "causal" if w.causal else "none"
+    if w.key_len_range:
+        mask = f"key_len~U[{w.key_len_range[0]},{w.key_len_range[1]}]"
+    return {"workload": w.name, "B": w.B, "H": w.H, "N_q": w.Nq, "N_k": w.Nk, "d": w.d,
+            "mask": mask, "scale": w.scale, "value_dist": f"N(0,{w.sigma}^2) bf16",
+            "seed": w.seed, "l2": l2_note, "parallelism": parallelism}
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, bounded row sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w)
+    per_step_s = float(os.environ.get("FA_REFERENCE_STEP_SECONDS", "2.0"))
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, x, per_step_s / 4, rng_seed=1)
+    rates, times, rows_used, cores = [], [], 0, 1
+    for i in range(args.steps):
+        r, n, t, cores = oracle_sample_rate(w, x, per_step_s, rng_seed=100 + i)
+        rates.append(r)
+        times.append(t)
+        rows_used += n
+    value = float(np.mean(rates))
+    ms = 1000.0 * w.flop / (value * 1e12)   # time the oracle would take for one whole step
+    sample = (f"{rows_used} random query rows of {w.B * w.H * w.Nq} over {args.steps} steps "
+              f"(~{per_step_s:.1f} s of CPU each), fp64, all keys each row sees")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, "n/a (CPU)", "host cores"), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the per-workload table, e2e and CPU baseline (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    from io_aware_exact_24_b200 import FA_OK, build, fa_get_device_status, load_library
+    build.build()
+    load_library()
+
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w)
+    clocks = ClockSampler(local)
+    ms, per, clk = time_device(w, x, args.steps, args.warmup, device, rank, world, clocks)
+    status = fa_get_device_status()
+    if status != FA_OK:
+        raise SystemExit(f"device status {status} after the timed region")
+    t_total = torch.tensor([sum(per)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t_total, op=torch.distributed.ReduceOp.MAX)
+    job_ms = float(t_total.item())
+    value = world * args.steps * w.flop / (job_ms / 1000.0) / 1e12
+
+    peaks, peaks_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = w.flop / (ms / 1000.0) / 1e12
+    traffic = load_traffic(w.name)
+    inputs_mb = 2 * w.B * w.H * (w.Nq + 2 * w.Nk) * w.d / 1e6
+    l2_note = (f"flushed between timed launches (256 MiB write outside the events); "
+               f"inputs {inputs_mb:.0f} MB")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": job_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, l2_note, f"replicas x{world}" if world > 1 else "single GPU"),
+        "pct_of_nominal_bf16_peak": 100.0 * achieved / NOMINAL_BF16_TFLOPS,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peaks_src} bf16_tflops (burst: kernel timed alone)",
+                     "kernel": f"fa_fwd_sm100_kernel<{w.d}>",
+                     "algorithmic_flop_per_launch": w.flop,
+                     "algorithmic_bytes_per_launch": w.algorithmic_bytes},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_extras:
+        e2e_ms, h2d, d2h = time_e2e(w, x, max(3, args.steps // 4), 3, device)
+        line["e2e"] = {"value": w.flop / (e2e_ms / 1000.0) / 1e12, "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_ms, "entry": "fa_fwd_host (pinned host buffers)"}
+        per_wl = {}
+        for name in WORKLOAD_ORDER:
+            wn = WORKLOADS[name]
+            xn = x if name == w.name else make_inputs(wn)
+            ms_n, _, _ = time_device(wn, xn, args.steps, args.warmup, device, 0, 1)
+            per_wl[name] = {"ms": ms_n, "tflops": wn.flop / (ms_n / 1000.0) / 1e12,
+                            "frac_of_peak": wn.flop / (ms_n / 1000.0) / 1e12 / peak,
+                            "algorithmic_gbs": wn.algorithmic_bytes / (ms_n / 1000.0) / 1e9}
+        line["per_workload"] = per_wl
+        cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
+        rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} random query rows of {w.B * w.H * w.Nq} "
+                                          f"({t:.1f} s), fp64, all keys each row sees"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

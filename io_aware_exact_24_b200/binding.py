@@ -62,6 +62,8 @@ def load_library() -> ctypes.CDLL:
             lib.fa_status_string.restype = ctypes.c_char_p
             lib.fa_get_device_status.argtypes = [vp]
             lib.fa_get_device_status.restype = i32
+            lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
+            lib.fa_selftest_wait_timeout.restype = i32
             lib.fa_version.argtypes = []
             lib.fa_version.restype = i32
             _lib = lib
@@ -128,6 +130,11 @@ def fa_fwd_host(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, wor
 
 def fa_get_device_status(stream=None) -> int:
     return int(load_library().fa_get_device_status(_stream(stream)))
+
+
+def fa_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:
+    """``fa_selftest_wait_timeout`` of include/fa.h (bounded-wait self test)."""
+    return int(load_library().fa_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
 
 
 def attention(q, k, v, causal=False, key_lens=None, scale=None, stream=None):

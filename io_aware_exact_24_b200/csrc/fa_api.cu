@@ -1,0 +1,284 @@
+// fa_api.cu -- host side of the C ABI declared in include/fa.h.
+//
+// Validates arguments (before any CUDA call), encodes the TMA tensor maps
+// for Q, K, V and O, and launches the sm_100a kernel.  No allocation, no
+// per-call state: the only caches are the driver's tensor-map encoder entry
+// point and a per-device "kernel attributes set" flag.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr unsigned long long kWaitLimitCycles = 1ull << 31;  // ~1 s at B200 clocks
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct DeviceState {
+    std::once_flag once;
+    int status = FA_OK;
+};
+DeviceState g_dev[kMaxDevices];
+
+// Per device, once: check the architecture and raise the kernels' shared-memory limit.
+int prepare_device(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    DeviceState& st = g_dev[dev];
+    std::call_once(st.once, [&] {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            st.status = FA_ERR_CUDA;
+            return;
+        }
+        if (major != 10 || minor != 0) {  // built for sm_100a only
+            st.status = FA_ERR_UNSUPPORTED;
+            return;
+        }
+        if (cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fa::Cfg<64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fa::Cfg<128>::kSmemBytes) != cudaSuccess) {
+            st.status = FA_ERR_CUDA;
+            return;
+        }
+        st.status = FA_OK;
+    });
+    return st.status;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Argument checks shared by fa_fwd and fa_fwd_host (no CUDA calls).
+int validate(const void* q, const void* k, const void* v, const void* o, const void* lse, int B, int H,
+             int N_q, int N_k, int d, float scale, const void* key_lens, bool* empty) {
+    if (B < 0 || H < 0 || N_q < 0 || N_k < 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (!(scale * 1.4426950408889634f > 0.f) || !std::isfinite(scale * 1.4426950408889634f))
+        return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    *empty = (B == 0 || H == 0 || N_q == 0);
+    if (*empty) return FA_OK;
+    if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;
+    // TMA: global strides must stay below 2^40 bytes.
+    const unsigned long long head_bytes_q = (unsigned long long)N_q * d * 2;
+    const unsigned long long head_bytes_k = (unsigned long long)N_k * d * 2;
+    if ((unsigned long long)H * head_bytes_q >= (1ull << 40) || (unsigned long long)H * head_bytes_k >= (1ull << 40))
+        return FA_ERR_UNSUPPORTED;
+    if (q == nullptr || o == nullptr || lse == nullptr) return FA_ERR_INVALID_ARG;
+    if (N_k > 0 && (k == nullptr || v == nullptr)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_MISALIGNED;
+    if (N_k > 0 && (!aligned(k, 16) || !aligned(v, 16))) return FA_ERR_MISALIGNED;
+    if (key_lens != nullptr && !aligned(key_lens, 4)) return FA_ERR_MISALIGNED;
+    return FA_OK;
+}
+
+// [B,H,N,d] bf16 viewed as a 4-D tensor (d, N, H, B), box 64 x 128 x 1 x 1, 128B swizzle.
+bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d) {
+    EncodeTiledFn enc = encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2, (cuuint64_t)H * N * d * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)fa::kBlockM, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
+           float scale, int causal, const int32_t* key_lens, cudaStream_t stream) {
+    CUtensorMap tq, tk, tv, to;
+    // With no keys the K/V maps are never read; give them a valid 1-row shape.
+    const void* kp = N_k > 0 ? k : q;
+    const void* vp = N_k > 0 ? v : q;
+    const int nk_map = N_k > 0 ? N_k : 1;
+    const int b_kv = N_k > 0 ? B : 1, h_kv = N_k > 0 ? H : 1;
+    if (!encode_bhnd(&tq, q, B, H, N_q, D) || !encode_bhnd(&tk, kp, b_kv, h_kv, nk_map, D) ||
+        !encode_bhnd(&tv, vp, b_kv, h_kv, nk_map, D) || !encode_bhnd(&to, o, B, H, N_q, D))
+        return FA_ERR_CUDA;
+    fa::FwdParams p;
+    p.lse = lse;
+    p.key_lens = key_lens;
+    p.B = B;
+    p.H = H;
+    p.Nq = N_q;
+    p.Nk = N_k;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.wait_limit = kWaitLimitCycles;
+    const int rows_per_cta = fa::kBlockM * fa::kTilesPerCta;
+    dim3 grid((unsigned)((N_q + rows_per_cta - 1) / rows_per_cta), (unsigned)H, (unsigned)B);
+    fa::fa_fwd_sm100_kernel<D><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct HostLayout {
+    size_t q, k, v, o, lse, kl, total;
+};
+HostLayout host_layout(int B, int H, int N_q, int N_k, int d, int has_key_lens) {
+    HostLayout L{};
+    const size_t bh = (size_t)B * H;
+    size_t off = 0;
+    L.q = off;
+    off = round_up(off + bh * N_q * d * 2, 256);
+    L.k = off;
+    off = round_up(off + bh * N_k * d * 2, 256);
+    L.v = off;
+    off = round_up(off + bh * N_k * d * 2, 256);
+    L.o = off;
+    off = round_up(off + bh * N_q * d * 2, 256);
+    L.lse = off;
+    off = round_up(off + bh * N_q * 4, 256);
+    L.kl = off;
+    off = round_up(off + (has_key_lens ? (size_t)B * 4 : 0), 256);
+    L.total = off;
+    return L;
+}
+
+__global__ void selftest_wait_kernel(unsigned long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        fa::mbar_init(fa::smem_addr(&bar), 1);
+        abort_flag = 0;
+        fa::fence_mbar_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on this barrier: the wait must give up and record a timeout.
+    (void)fa::wait_bounded(fa::smem_addr(&bar), 0, &abort_flag, limit);
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k, int d,
+           float scale, int causal, const int32_t* key_lens, fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK || empty) return st;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s);
+}
+
+size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has_key_lens) {
+    if (B < 0 || H < 0 || N_q < 0 || N_k < 0 || (d != 64 && d != 128)) return 0;
+    return host_layout(B, H, N_q, N_k, d, has_key_lens).total;
+}
+
+int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
+                int d, float scale, int causal, const int32_t* key_lens, void* workspace, size_t workspace_bytes,
+                fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK || empty) return st;
+    const HostLayout L = host_layout(B, H, N_q, N_k, d, key_lens != nullptr);
+    if (workspace == nullptr || workspace_bytes < L.total) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    const size_t bh = (size_t)B * H;
+    const size_t q_bytes = bh * N_q * d * 2, kv_bytes = bh * N_k * d * 2;
+    if (cudaMemcpyAsync(ws + L.q, q, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return FA_ERR_CUDA;
+    if (kv_bytes > 0) {
+        if (cudaMemcpyAsync(ws + L.k, k, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(ws + L.v, v, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return FA_ERR_CUDA;
+    }
+    const int32_t* kl_dev = nullptr;
+    if (key_lens != nullptr) {
+        if (cudaMemcpyAsync(ws + L.kl, key_lens, (size_t)B * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return FA_ERR_CUDA;
+        kl_dev = reinterpret_cast<const int32_t*>(ws + L.kl);
+    }
+    st = fa_fwd(ws + L.q, N_k > 0 ? ws + L.k : nullptr, N_k > 0 ? ws + L.v : nullptr, ws + L.o,
+                reinterpret_cast<float*>(ws + L.lse), B, H, N_q, N_k, d, scale, causal, kl_dev, stream);
+    if (st != FA_OK) return st;
+    if (cudaMemcpyAsync(o, ws + L.o, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse, ws + L.lse, bh * N_q * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported configuration or device";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer misaligned";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
+        case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no CUDA device";
+        case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: kernel pipeline wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int fa_get_device_status(fa_stream_t stream) {
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return v == 0 ? FA_OK : v;
+}
+
+int fa_selftest_wait_timeout(unsigned long long limit_cycles, fa_stream_t stream) {
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    if (limit_cycles > (1ull << 32)) return FA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    return fa_get_device_status(stream);
+}
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

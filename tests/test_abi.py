@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from io_aware_exact_24_b200 import binding
+from io_aware_exact_24_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        names += re.findall(r"^FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("fa_fwd", "fa_fwd_host", "fa_fwd_host_workspace_size", "fa_status_string",
+                 "fa_get_device_status", "fa_version", "fa_selftest_wait_timeout"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(lib):
+    assert binding.fa_status_string(0) == "FA_OK"
+    for code in range(-6, 0):
+        assert binding.fa_status_string(code).startswith("FA_ERR_")
+    assert binding.fa_status_string(12345) == "unknown status"
+    assert binding.fa_version() == 10000
+
+
+# A fake, suitably aligned "device" address: validation must fail before it is used.
+P = 1 << 20
+
+
+def call(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0,
+         key_lens=None):
+    return binding.fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, key_lens,
+                          stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=256), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(H=-2), binding.FA_ERR_INVALID_ARG),
+    (dict(Nq=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(Nk=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=1e-46), binding.FA_ERR_INVALID_ARG),   # 0 once rounded to fp32
+    (dict(q=None), binding.FA_ERR_INVALID_ARG),
+    (dict(o=None), binding.FA_ERR_INVALID_ARG),
+    (dict(lse=None), binding.FA_ERR_INVALID_ARG),
+    (dict(k=None), binding.FA_ERR_INVALID_ARG),
+    (dict(v=None), binding.FA_ERR_INVALID_ARG),
+    (dict(q=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(k=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(v=P + 4), binding.FA_ERR_MISALIGNED),
+    (dict(o=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(lse=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(key_lens=P + 1), binding.FA_ERR_MISALIGNED),
+    (dict(B=70000), binding.FA_ERR_UNSUPPORTED),
+    (dict(H=65536), binding.FA_ERR_UNSUPPORTED),
+])
+def test_argument_errors_are_reported_before_any_cuda_call(lib, kw, code):
+    assert call(**kw) == code
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(Nq=0),
+                                dict(B=0, q=None, k=None, v=None, o=None, lse=None)])
+def test_empty_problems_are_noops(lib, kw):
+    assert call(**kw) == binding.FA_OK
+
+
+def test_no_keys_allows_null_k_v_until_the_device_check(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("would launch on fake addresses; covered by the GPU tests")
+    assert call(Nk=0, k=None, v=None) == binding.FA_ERR_NO_DEVICE
+
+
+def test_host_entry_validates_workspace(lib):
+    need = binding.fa_fwd_host_workspace_size(2, 3, 100, 50, 64, True)
+    assert need >= 2 * 3 * (100 + 2 * 50 + 100) * 64 * 2 + 2 * 3 * 100 * 4 + 8
+    assert need % 256 == 0
+    assert binding.fa_fwd_host_workspace_size(1, 1, 8, 8, 96, False) == 0
+    st = binding.fa_fwd_host(P, P, P, P, P, 1, 1, 8, 8, 64, 0.125, 0, None, P, 16,
+                             stream=0, check=False)
+    assert st == binding.FA_ERR_INVALID_ARG
+    need = binding.fa_fwd_host_workspace_size(1, 1, 8, 8, 64, False)
+    st = binding.fa_fwd_host(P, P, P, P, P, 1, 1, 8, 8, 64, 0.125, 0, None, P + 16, need,
+                             stream=0, check=False)
+    assert st == binding.FA_ERR_MISALIGNED
+
+
+def test_without_a_gpu_valid_calls_report_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call() == binding.FA_ERR_NO_DEVICE
+    assert binding.fa_get_device_status(0) == binding.FA_ERR_NO_DEVICE

@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Small and medium problems are compared element by element; the two
+full-size long-sequence workloads are compared on sampled rows the oracle
+evaluates one by one, plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from io_aware_exact_24_b200.inputs import (WORKLOADS, bf16_bits_to_f32, f32_to_bf16_bits,
+                                           make_inputs, normal_bf16)
+
+from fa_testutil import compare, run_fa
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from io_aware_exact_24_b200.build import build
+    build()
+
+
+def _rand(B, H, Nq, Nk, d, seed, sigma=1.0):
+    return (normal_bf16((B, H, Nq, d), seed, 0, sigma), normal_bf16((B, H, Nk, d), seed, 1, sigma),
+            normal_bf16((B, H, Nk, d), seed, 2, sigma))
+
+
+@pytest.mark.parametrize("name", ["tiny", "gpt2_causal_1k", "bert_padded_512"])
+def test_workload_full_compare(name):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    o, lse = run_fa(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    o_ref, lse_ref = oracle.attn_ref(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    errs = compare(o, lse, o_ref, lse_ref, name)
+    print(f"{name}: max|dO|={errs[0]:.3e} relF={errs[1]:.3e} max|dLSE|={errs[2]:.3e}")
+
+
+def _sample_rows(w, rng, per_head=12):
+    rows = []
+    edges = [0, 1, 127, 128, 255, 256, w.Nq - 129, w.Nq - 128, w.Nq - 65, w.Nq - 64, w.Nq - 2,
+             w.Nq - 1]
+    for bh in range(w.B * w.H):
+        pick = set(i for i in edges if 0 <= i < w.Nq)
+        pick.update(rng.integers(0, w.Nq, size=per_head).tolist())
+        rows += [bh * w.Nq + i for i in sorted(pick)]
+    return np.array(rows, np.int64)
+
+
+@pytest.mark.parametrize("name", ["long_16k_d64", "causal_8000_d128"])
+def test_workload_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    o, lse = run_fa(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    rows = _sample_rows(w, np.random.default_rng(123))
+    o_ref, lse_ref = oracle.attn_ref_rows(x["q"], x["k"], x["v"], w.scale, rows, w.causal,
+                                          x["key_lens"])
+    errs = compare(o.reshape(-1, w.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, name)
+    print(f"{name} ({rows.size} rows): max|dO|={errs[0]:.3e} relF={errs[1]:.3e} "
+          f"max|dLSE|={errs[2]:.3e}")
+    # properties at full size: |O| is bounded by max|V| (convex combination of V rows)
+    vmax = np.abs(bf16_bits_to_f32(x["v"])).max()
+    assert np.abs(o).max() <= vmax * (1 + 2**-7)
+
+
+EDGE = [
+    # B, H, Nq, Nk, d, causal, key_lens
+    (1, 1, 1, 1, 64, False, None),
+    (1, 1, 1, 1, 128, True, None),
+    (1, 2, 2, 2, 64, True, None),
+    (1, 1, 63, 63, 64, False, None),
+    (1, 1, 64, 64, 128, True, None),
+    (2, 1, 127, 127, 64, True, None),
+    (1, 1, 129, 129, 128, False, None),
+    (1, 2, 255, 255, 64, True, None),
+    (1, 1, 256, 256, 128, True, None),
+    (1, 1, 257, 257, 64, True, None),
+    (2, 2, 300, 300, 128, False, None),
+    (1, 1, 100, 300, 64, True, None),      # Nq < Nk: bottom-right causal
+    (1, 1, 300, 100, 128, True, None),     # Nq > Nk: leading rows see no key
+    (1, 1, 513, 129, 64, True, None),      # whole Q tiles with no visible key
+    (1, 3, 200, 333, 64, False, None),
+    (3, 2, 140, 140, 64, False, [0, 1, 140]),
+    (4, 1, 260, 260, 128, True, [0, 129, 1000, -5]),
+    (2, 2, 384, 384, 64, False, [128, 255]),
+    (1, 1, 64, 0, 64, False, None),        # no keys at all
+    (2, 1, 200, 0, 128, True, None),
+    (2, 3, 1000, 1000, 128, True, None),   # several tiles, ragged tail
+    (1, 2, 1100, 900, 64, False, [700]),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[str(c[:6]) + ("kl" if c[6] else "") for c in EDGE])
+def test_edge_cases(case):
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 31 + Nq + Nk + d)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    out = {}
+    o, lse = run_fa(q, k, v, 1.0 / np.sqrt(d), causal, kl_arr, o_guard=4096, out=out)
+    assert out["guards_ok"], "wrote outside O / LSE"
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, 1.0 / np.sqrt(d), causal, kl_arr)
+    compare(o, lse, o_ref, lse_ref, str(case))
+
+
+def test_empty_problems_touch_nothing():
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd
+    o = torch.full((4,), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((4,), 5.0, dtype=torch.float32, device="cuda")
+    for B, H, Nq in ((0, 2, 8), (2, 0, 8), (2, 2, 0)):
+        fa_fwd(o, o, o, o, lse, B, H, Nq, 8, 64, 0.125)
+    torch.cuda.synchronize()
+    assert (o == 3.0).all() and (lse == 5.0).all()
+
+
+def test_deterministic_bitwise():
+    q, k, v = _rand(2, 4, 700, 700, 128, 77)
+    a, b = {}, {}
+    run_fa(q, k, v, 0.09, True, None, out=a)
+    run_fa(q, k, v, 0.09, True, None, out=b)
+    assert np.array_equal(a["o_bits"], b["o_bits"])
+    assert np.array_equal(a["lse_raw"].view(np.uint32), b["lse_raw"].view(np.uint32))
+
+
+def test_masked_garbage_is_invisible_bitwise():
+    B, H, N, d = 2, 2, 400, 64
+    q, k, v = _rand(B, H, N, N, d, 78)
+    kl = np.array([150, 333], np.int32)
+    a, b = {}, {}
+    run_fa(q, k, v, 0.125, True, kl, out=a)
+    k2, v2 = k.copy(), v.copy()
+    for bb in range(B):
+        k2[bb, :, kl[bb]:] = f32_to_bf16_bits(np.float32(8192.0))
+        v2[bb, :, kl[bb]:] = f32_to_bf16_bits(np.float32(-8192.0))
+    run_fa(q, k2, v2, 0.125, True, kl, out=b)
+    assert np.array_equal(a["o_bits"], b["o_bits"])
+    assert np.array_equal(a["lse_raw"].view(np.uint32), b["lse_raw"].view(np.uint32))
+
+
+def test_single_visible_key_is_exact():
+    # causal row 0 and a key_len of 1 see one key: P = 1 exactly, O = V_0 bit for bit
+    B, H, N, d = 2, 2, 300, 128
+    q, k, v = _rand(B, H, N, N, d, 79)
+    o, _ = run_fa(q, k, v, 0.1, True, None)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    assert np.array_equal(o[:, :, 0, :], vf[:, :, 0, :])
+    o1, _ = run_fa(q, k, v, 0.1, False, np.array([1, 1], np.int32))
+    assert np.array_equal(o1, np.broadcast_to(vf[:, :, :1, :], o1.shape))
+
+
+def test_zero_query_gives_mean_of_values():
+    B, H, N, d = 1, 2, 520, 64
+    _, k, v = _rand(B, H, N, N, d, 80)
+    q = np.zeros((B, H, N, d), np.uint16)
+    o, lse = run_fa(q, k, v, 0.125, True, None)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    means = np.cumsum(vf, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, means, rtol=0, atol=1.5e-2)
+    np.testing.assert_allclose(lse, np.log(np.arange(1, N + 1))[None, None, :].repeat(H, 1),
+                               rtol=0, atol=1e-3)
+
+
+def test_host_entry_matches_device_entry():
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd_host, fa_fwd_host_workspace_size
+    B, H, Nq, Nk, d = 2, 3, 333, 257, 128
+    q, k, v = _rand(B, H, Nq, Nk, d, 81)
+    kl = np.array([200, 257], np.int32)
+    dev = {}
+    run_fa(q, k, v, 0.088, True, kl, out=dev)
+    ws_bytes = fa_fwd_host_workspace_size(B, H, Nq, Nk, d, True)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    o = np.empty((B, H, Nq, d), np.uint16)
+    lse = np.empty((B, H, Nq), np.float32)
+    fa_fwd_host(q, k, v, o, lse, B, H, Nq, Nk, d, 0.088, True, kl, ws, ws_bytes)
+    assert np.array_equal(o.view(np.int16), dev["o_bits"])
+    assert np.array_equal(lse.view(np.uint32), dev["lse_raw"].view(np.uint32))
+
+
+def test_device_status_is_clean_after_the_suite():
+    from io_aware_exact_24_b200 import FA_OK, fa_get_device_status
+    assert fa_get_device_status() == FA_OK
