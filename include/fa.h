@@ -142,6 +142,13 @@ FA_API int fa_get_device_status(fa_stream_t stream);
  */
 FA_API int fa_selftest_wait_timeout(unsigned long long limit_cycles, fa_stream_t stream);
 
+/*
+ * fa_last_error -- the CUDA call and error text behind the most recent
+ * FA_ERR_CUDA returned on the calling thread ("" if none).  The string
+ * belongs to the library and stays valid until the thread's next failing call.
+ */
+FA_API const char *fa_last_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 FA_API int fa_version(void);
 

@@ -31,7 +31,9 @@ class FaError(RuntimeError):
 
     def __init__(self, status: int, where: str):
         self.status = int(status)
-        super().__init__(f"{where}: {fa_status_string(status)} (status {status})")
+        detail = fa_last_error() if status == FA_ERR_CUDA else ""
+        super().__init__(f"{where}: {fa_status_string(status)} (status {status})"
+                         + (f": {detail}" if detail else ""))
 
 
 def library_path() -> str:
@@ -64,6 +66,8 @@ def load_library() -> ctypes.CDLL:
             lib.fa_get_device_status.restype = i32
             lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
             lib.fa_selftest_wait_timeout.restype = i32
+            lib.fa_last_error.argtypes = []
+            lib.fa_last_error.restype = ctypes.c_char_p
             lib.fa_version.argtypes = []
             lib.fa_version.restype = i32
             _lib = lib
@@ -94,6 +98,10 @@ def _stream(stream) -> int | None:
 
 def fa_status_string(status: int) -> str:
     return load_library().fa_status_string(int(status)).decode()
+
+
+def fa_last_error() -> str:
+    return load_library().fa_last_error().decode()
 
 
 def fa_version() -> int:

@@ -9,6 +9,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -18,6 +19,14 @@
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
+
+// Last FA_ERR_CUDA cause on this thread (what fa_last_error returns).
+thread_local char t_last_error[256] = "";
+
+int cuda_fail(const char* what, cudaError_t e) {
+    snprintf(t_last_error, sizeof t_last_error, "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+    return FA_ERR_CUDA;
+}
 constexpr unsigned long long kWaitLimitCycles = 1ull << 31;  // ~1 s at B200 clocks
 constexpr int kMaxDevices = 64;
 
@@ -51,20 +60,23 @@ int prepare_device(int dev) {
     DeviceState& st = g_dev[dev];
     std::call_once(st.once, [&] {
         int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-            st.status = FA_ERR_CUDA;
+        cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e != cudaSuccess) {
+            st.status = cuda_fail("cudaDeviceGetAttribute", e);
             return;
         }
         if (major != 10 || minor != 0) {  // built for sm_100a only
             st.status = FA_ERR_UNSUPPORTED;
             return;
         }
-        if (cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fa::Cfg<64>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fa::Cfg<128>::kSmemBytes) != cudaSuccess) {
-            st.status = FA_ERR_CUDA;
+        e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fa::Cfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::Cfg<128>::kSmemBytes);
+        if (e != cudaSuccess) {
+            st.status = cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
             return;
         }
         st.status = FA_OK;
@@ -121,8 +133,10 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     const int nk_map = N_k > 0 ? N_k : 1;
     const int b_kv = N_k > 0 ? B : 1, h_kv = N_k > 0 ? H : 1;
     if (!encode_bhnd(&tq, q, B, H, N_q, D) || !encode_bhnd(&tk, kp, b_kv, h_kv, nk_map, D) ||
-        !encode_bhnd(&tv, vp, b_kv, h_kv, nk_map, D) || !encode_bhnd(&to, o, B, H, N_q, D))
+        !encode_bhnd(&tv, vp, b_kv, h_kv, nk_map, D) || !encode_bhnd(&to, o, B, H, N_q, D)) {
+        snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
         return FA_ERR_CUDA;
+    }
     fa::FwdParams p;
     p.lse = lse;
     p.key_lens = key_lens;
@@ -133,10 +147,11 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.wait_limit = kWaitLimitCycles;
-    const int rows_per_cta = fa::kBlockM * fa::kTilesPerCta;
+    const int rows_per_cta = fa::kBlockM;
     dim3 grid((unsigned)((N_q + rows_per_cta - 1) / rows_per_cta), (unsigned)H, (unsigned)B);
     fa::fa_fwd_sm100_kernel<D><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -193,7 +208,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
         cudaGetLastError();
         return FA_ERR_NO_DEVICE;
     }
-    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     st = prepare_device(dev);
     if (st != FA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -219,25 +235,23 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse
     char* ws = static_cast<char*>(workspace);
     const size_t bh = (size_t)B * H;
     const size_t q_bytes = bh * N_q * d * 2, kv_bytes = bh * N_k * d * 2;
-    if (cudaMemcpyAsync(ws + L.q, q, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return FA_ERR_CUDA;
-    if (kv_bytes > 0) {
-        if (cudaMemcpyAsync(ws + L.k, k, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-            cudaMemcpyAsync(ws + L.v, v, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return FA_ERR_CUDA;
-    }
+    cudaError_t e = cudaMemcpyAsync(ws + L.q, q, q_bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && kv_bytes > 0) e = cudaMemcpyAsync(ws + L.k, k, kv_bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && kv_bytes > 0) e = cudaMemcpyAsync(ws + L.v, v, kv_bytes, cudaMemcpyHostToDevice, s);
     const int32_t* kl_dev = nullptr;
-    if (key_lens != nullptr) {
-        if (cudaMemcpyAsync(ws + L.kl, key_lens, (size_t)B * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return FA_ERR_CUDA;
+    if (e == cudaSuccess && key_lens != nullptr) {
+        e = cudaMemcpyAsync(ws + L.kl, key_lens, (size_t)B * 4, cudaMemcpyHostToDevice, s);
         kl_dev = reinterpret_cast<const int32_t*>(ws + L.kl);
     }
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (host to device)", e);
     st = fa_fwd(ws + L.q, N_k > 0 ? ws + L.k : nullptr, N_k > 0 ? ws + L.v : nullptr, ws + L.o,
                 reinterpret_cast<float*>(ws + L.lse), B, H, N_q, N_k, d, scale, causal, kl_dev, stream);
     if (st != FA_OK) return st;
-    if (cudaMemcpyAsync(o, ws + L.o, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse, ws + L.lse, bh * N_q * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return FA_ERR_CUDA;
-    return cudaStreamSynchronize(s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    e = cudaMemcpyAsync(o, ws + L.o, q_bytes, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(lse, ws + L.lse, bh * N_q * 4, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (device to host)", e);
+    e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? FA_OK : cuda_fail("cudaStreamSynchronize", e);
 }
 
 const char* fa_status_string(int status) {
@@ -259,11 +273,14 @@ int fa_get_device_status(fa_stream_t stream) {
         cudaGetLastError();
         return FA_ERR_NO_DEVICE;
     }
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    e = cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyFromSymbol(status)", e);
     const int zero = 0;
-    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyToSymbol(status)", e);
     return v == 0 ? FA_OK : v;
 }
 
@@ -275,9 +292,12 @@ int fa_selftest_wait_timeout(unsigned long long limit_cycles, fa_stream_t stream
     }
     if (limit_cycles > (1ull << 32)) return FA_ERR_INVALID_ARG;
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("self-test kernel launch", e);
     return fa_get_device_status(stream);
 }
+
+const char* fa_last_error(void) { return t_last_error; }
 
 int fa_version(void) { return kVersion; }
 

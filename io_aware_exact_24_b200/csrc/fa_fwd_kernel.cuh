@@ -8,29 +8,30 @@
 // matrix is never stored).  The pages' kernels target A100/RTX 3090/T4 and
 // Hopper; this one is laid out for Blackwell:
 //
-//  * one CTA = one (b, h) and two 128-row Q tiles (256 query rows) that share
-//    every K/V tile loaded into shared memory;
-//  * warp 8 (one elected lane) streams Q once and then K_j, V_j through a ring
-//    of shared-memory slots with TMA (128B-swizzled boxes of 64 columns x 128
-//    rows), one mbarrier pair (full/empty) per slot -- the double buffering
-//    that "FlashAttention：把注意力从公式写成数据流" (section "端侧与专用加速器")
-//    names for hiding loads;
-//  * warp 9 (one elected lane) issues tcgen05 MMAs: S_t = Q_t K_j^T into TMEM
-//    (fp32, 128 lanes x 128 columns) and O_t += P_t V_j with P_t read from
-//    TMEM and V_j from shared memory; completions are signalled with
-//    tcgen05.commit onto mbarriers;
-//  * warps 0-3 own Q tile 0 and warps 4-7 own Q tile 1 (one thread per query
-//    row, because TMEM lane i is row i): load the S row from TMEM, mask it on
-//    boundary tiles only, update the running max m and sum l in the exp2
-//    domain, write P back to TMEM as bf16, and rescale their O row in TMEM
-//    when the max moved by more than 2^8 (exact: m, l and O always share one
-//    reference max);
-//  * while one tile's rows are in softmax the tensor core works on the other
-//    tile, so the MMAs of tile 1 overlap the exponentials of tile 0 and back;
-//  * epilogue: O / l -> bf16 into the (now idle) Q buffer, TMA store clipped at
-//    N_q; LSE = ln2 * (m + log2 l); rows without a visible key give O = 0 and
-//    LSE = -inf ("FlashAttention：把注意力从公式写成数据流", section "精度、掩码和
-//    边界情况": masked positions never enter the normaliser).
+//  * one CTA = one (b, h) and one 128-row Q tile (TMEM lane i = query row i);
+//  * warp 8 (one elected lane) loads Q once and then streams K and V tiles
+//    (128 keys) through a ring of shared-memory slots with TMA (128B-swizzled
+//    boxes of 64 columns x 128 rows), one full/empty mbarrier pair per slot --
+//    the double buffering "FlashAttention：把注意力从公式写成数据流" (section
+//    "端侧与专用加速器") names for hiding loads;
+//  * warp 9 (one elected lane) issues the tcgen05 MMAs.  S is double-buffered
+//    in TMEM: S(j+2) = Q K_{j+2}^T is issued right after O += P(j) V_j, so the
+//    score tile the softmax needs next is computed while it works on the
+//    current one and the softmax never waits on the tensor core;
+//  * warps 0-7 do the online softmax, one thread per query row and tile:
+//    warps q and q+4 both own TMEM lanes 32q..32q+31 and take the K/V tiles
+//    in turn (even / odd), so one warp's exponentials overlap the other's
+//    loads and maxima.  Only the running reference max passes between them
+//    (shared memory + an mbarrier); each keeps its own partial row sum.
+//    Exponentials are taken in the exp2 domain, some on MUFU and some with a
+//    polynomial on the FMA pipe; P goes back to TMEM as bf16 over the first
+//    half of the tile's S buffer and feeds the PV MMA from there;
+//  * the reference max moves only when the row max grows by more than 2^8;
+//    O is then rescaled in TMEM (exact: m, l and O always share one max);
+//  * epilogue: O / l -> bf16 -> shared memory (128B-swizzled) -> TMA store
+//    clipped at N_q; LSE = ln2 * (m + log2 l); rows without a visible key give
+//    O = 0 and LSE = -inf ("FlashAttention：把注意力从公式写成数据流", section
+//    "精度、掩码和边界情况": masked positions never enter the normaliser).
 //
 // Every mbarrier wait is bounded; a wait that runs out records
 // FA_ERR_DEVICE_TIMEOUT in g_fa_status and the CTA winds down instead of
@@ -42,20 +43,29 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa {
 
-constexpr int kBlockM = 128;        // query rows per Q tile (= TMEM lanes)
+constexpr int kBlockM = 128;        // query rows per CTA (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
-constexpr int kTilesPerCta = 2;     // Q tiles sharing one K/V stream
-constexpr int kNumThreads = 320;    // 8 softmax warps + producer warp + MMA warp
+constexpr int kNumThreads = 384;    // 8 softmax warps, producer, MMA, 2 spare
+constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
+// Registers are allocated per warpgroup: 384 threads x 168 at launch, then the
+// softmax warpgroups take 216 and the producer/MMA warpgroup keeps 72
+// (2*128*216 + 128*72 = 384*168).
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 72;
 constexpr int kSwizzleBoxBytes = 128 * 128;  // one 64-column x 128-row bf16 box
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only if max grows > 2^8
 constexpr int kStatusTimeout = -6;           // FA_ERR_DEVICE_TIMEOUT
+// named barriers (epilogue only): 1..4 pair the two warps of a lane quadrant, 5 spans all softmax warps
+constexpr uint32_t kBarQuadBase = 1;
+constexpr uint32_t kBarSoftmaxAll = 5;
 
 struct FwdParams {
     float* lse;                 // [B,H,Nq]
@@ -71,22 +81,28 @@ struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kBoxes = D / 64;                        // 64-column boxes per row
     static constexpr int kTileBytes = kBlockM * D * 2;           // one Q / K / V tile
-    static constexpr int kStages = (D == 64) ? 8 : 4;            // K/V ring slots
+    static constexpr int kStages = (D == 64) ? 10 : 5;           // K/V ring slots
+    // Of every 8 pairs of probabilities, this many are computed on the FMA pipe
+    // (exp2_fma2) and the rest on MUFU, so neither unit is the lone bottleneck.
+#ifdef FA_EMU_PAIRS_D64
+    static constexpr int kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
+#else
+    static constexpr int kEmuPairs = 2;
+#endif
     static constexpr int kQOff = 0;
-    static constexpr int kKvOff = kTilesPerCta * kTileBytes;
+    static constexpr int kKvOff = kTileBytes;
     static constexpr int kBarOff = kKvOff + kStages * kTileBytes;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
-    static constexpr int kNumBars = 8 + 2 * kStages;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;      // + alignment slack
-    // TMEM columns
-    static constexpr uint32_t kColS0 = 0;
-    static constexpr uint32_t kColO0 = 256;
-    __host__ __device__ static constexpr uint32_t col_s(int t) { return kColS0 + 128u * t; }
-    __host__ __device__ static constexpr uint32_t col_o(int t) { return kColO0 + (uint32_t)D * t; }
-    // P (bf16, 64 columns): separate columns when they fit, else over the first
-    // half of the tile's own S columns (S is fully read before P is written).
-    __host__ __device__ static constexpr uint32_t col_p(int t) { return D == 64 ? 384u + 64u * t : col_s(t); }
+    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
+    // m_ready[4 quadrants][2 parities], drain
+    static constexpr int kNumBars = 16 + 2 * kStages;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
+    static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [parity][row]
+    static constexpr int kEpiOff = kMrefOff + 2 * kBlockM * 4;   // epilogue exchange: m [2][row], l [2][row]
+    static constexpr int kSmemBytes = kEpiOff + 4 * kBlockM * 4 + 1024;  // + alignment slack
+    // TMEM columns: S buffers at 0 and 128 (P of a tile over the first 64
+    // columns of its S buffer), O at 256.
+    __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
+    static constexpr uint32_t kColO = 256;
     // Instruction descriptors (kind::f16): D=f32, A=B=bf16, M=128.
     //   QK^T: A=Q K-major, B=K K-major, N=128.  PV: A=P (TMEM, K-major), B=V MN-major, N=D.
     static constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
@@ -118,7 +134,9 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        // sleeps until the phase completes (or 0.1 ms passes): a waiting warp
+        // leaves its issue slots to the warps that are computing
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if (*abort_flag) return false;
         if ((unsigned long long)(clock64() - t0) > limit) {
             *abort_flag = 1;
@@ -126,6 +144,64 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
             return false;
         }
     }
+}
+
+// 2^x for two finite x on the FMA pipe: x = n + r with n = rint(x) (added into the
+// exponent field) and 2^r, r in [-1/2, 1/2], from the fitted cubic in exp2_poly.cuh.
+// x is clamped at -125 so 2^n stays a normal number; callers never pass -inf.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));  // 1.5*2^23: rint in the low bits
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 r = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(r, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+    q = __ffma2_rn(q, r, make_float2(kExp2C1, kExp2C1));
+    q = __ffma2_rn(q, r, make_float2(kExp2C0, kExp2C0));
+    float2 e;
+    e.x = __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23));
+    e.y = __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23));
+    return e;
+}
+
+// p = 2^(s*c - mu) for keys 64*h2 .. 64*h2+63 of the thread's row, packed to
+// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2; the fp32 p are
+// summed into (l0, l1).  kEmu of every 8 pairs go through exp2_fma2, the rest
+// through MUFU ex2 (which maps -inf to 0, so masked tiles use kEmu = 0).
+template <int kEmu, int h2>
+__device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float c, float mu, uint32_t taddr_p,
+                                               float2& l0, float2& l1) {
+    const float2 c2 = make_float2(c, c);
+    const float2 nmu = make_float2(-mu, -mu);
+    uint32_t w[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int pi = 32 * h2 + i;
+        const float2 x = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), c2, nmu);
+        float2 e;
+        if ((i & 7) < kEmu) {
+            e = exp2_fma2(x);
+        } else {
+            e.x = ex2_approx(x.x);
+            e.y = ex2_approx(x.y);
+        }
+        if (i & 1)
+            l1 = __fadd2_rn(l1, e);
+        else
+            l0 = __fadd2_rn(l0, e);
+        w[i] = pack_bf16x2(e.x, e.y);
+    }
+    tmem_st32(taddr_p + 32u * h2, w);
+}
+
+// Maximum of s[o .. o+31] as a tree of three-input max (depth 4).
+__device__ __forceinline__ float chunk_max32(const float (&s)[kBlockN], int o) {
+    float a[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) a[i] = max3f(s[o + 3 * i], s[o + 3 * i + 1], s[o + 3 * i + 2]);
+    a[10] = fmaxf(s[o + 30], s[o + 31]);
+    const float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]), b2 = max3f(a[6], a[7], a[8]);
+    return max3f(max3f(b0, b1, b2), a[9], a[10]);
 }
 
 // Number of keys (prefix length) a query row may see.
@@ -150,44 +226,36 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t bar_q_full = base + C::kBarOff;
     auto bar_kv_full = [&](int s) { return base + C::kBarOff + 8u * (1 + s); };
     auto bar_kv_empty = [&](int s) { return base + C::kBarOff + 8u * (1 + C::kStages + s); };
-    auto bar_s_full = [&](int t) { return base + C::kBarOff + 8u * (1 + 2 * C::kStages + t); };
-    auto bar_p_full = [&](int t) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + t); };
-    auto bar_o_full = [&](int t) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + t); };
-    const uint32_t bar_drain = base + C::kBarOff + 8u * (7 + 2 * C::kStages);
+    auto bar_s_full = [&](int b) { return base + C::kBarOff + 8u * (1 + 2 * C::kStages + b); };
+    auto bar_p_full = [&](int b) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + b); };
+    auto bar_o_done = [&](int b) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + b); };
+    auto bar_m_ready = [&](int qd, int b) { return base + C::kBarOff + 8u * (7 + 2 * C::kStages + 2 * qd + b); };
+    const uint32_t bar_drain = base + C::kBarOff + 8u * (15 + 2 * C::kStages);
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
-    auto q_tile = [&](int t) { return base + C::kQOff + (uint32_t)(t * C::kTileBytes); };
+    float* const mref = reinterpret_cast<float*>(base_ptr + C::kMrefOff);     // [parity][row]
+    float* const epi = reinterpret_cast<float*>(base_ptr + C::kEpiOff);       // m [2][row], l [2][row]
+    const uint32_t q_tile = base + C::kQOff;
     auto kv_slot = [&](int s) { return base + C::kKvOff + (uint32_t)(s * C::kTileBytes); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work item: (b, h, 256-row block); heavy causal blocks launch first
+    // ---- work item: (b, h, 128-row block); heavy causal blocks launch first
     const int num_m = (int)gridDim.x;
     const int m_blk = p.causal ? (num_m - 1 - (int)blockIdx.x) : (int)blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
-    const int m0 = m_blk * (kTilesPerCta * kBlockM);
+    const int m0 = m_blk * kBlockM;
     int kl = p.Nk;
     if (p.key_lens != nullptr) {
         kl = p.key_lens[b];
         kl = kl < 0 ? 0 : (kl > p.Nk ? p.Nk : kl);
     }
     const int off = p.Nk - p.Nq;  // causal diagonal offset (bottom-right aligned)
-    // K/V tiles each Q tile must visit (0 for a tile with no query row).
-    int n_tiles[kTilesPerCta];
-#pragma unroll
-    for (int t = 0; t < kTilesPerCta; ++t) {
-        const int first = m0 + t * kBlockM;
-        if (first >= p.Nq) {
-            n_tiles[t] = 0;
-            continue;
-        }
-        const int last = min(first + kBlockM - 1, p.Nq - 1);
-        const int n_end = row_key_limit(last, kl, off, p.causal);
-        n_tiles[t] = (n_end + kBlockN - 1) / kBlockN;
-    }
-    const int n_kv = max(n_tiles[0], n_tiles[1]);
+    // K/V tiles this Q tile must visit: enough for its last real row.
+    const int last_row = min(m0 + kBlockM - 1, p.Nq - 1);
+    const int n_kv = (row_key_limit(last_row, kl, off, p.causal) + kBlockN - 1) / kBlockN;
 
     // ---- setup: barriers (producer lane 0), TMEM (MMA warp)
     if (warp == kProducerWarp && lane == 0) {
@@ -196,11 +264,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             mbar_init(bar_kv_full(s), 1);
             mbar_init(bar_kv_empty(s), 1);
         }
-        for (int t = 0; t < kTilesPerCta; ++t) {
-            mbar_init(bar_s_full(t), 1);
-            mbar_init(bar_p_full(t), kBlockM);
-            mbar_init(bar_o_full(t), 1);
+        mbar_init(bar_s_full(0), 1);
+        mbar_init(bar_s_full(1), 1);
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(bar_p_full(b2), kSoftmaxWarps / 2);
+            mbar_init(bar_o_done(b2), 1);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(bar_m_ready(i >> 1, i & 1), 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -218,41 +288,38 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == kProducerWarp) {
+    // The K/V load order, shared by producer and MMA issuer: K0, K1, then for
+    // every j: V_j followed by K_{j+2} -- the order the MMAs consume them in.
+    if (warp >= kProducerWarp) {
+      setmaxnreg_dec<kRegsControl>();   // whole warpgroup 2, one instruction
+      if (warp == kProducerWarp) {
         // =========================================================== TMA producer
         if (lane == 0 && n_kv > 0) {
             const uint64_t pol_kv = policy_evict_last();
             const uint64_t pol_q = policy_evict_first();
-            // only tiles with work are loaded: a tile that sees no key writes its
-            // zeros through the same buffer, which must not have a copy in flight
-            int q_tiles = 0;
-            for (int t = 0; t < kTilesPerCta; ++t) q_tiles += (n_tiles[t] > 0) ? 1 : 0;
-            mbar_arrive_expect_tx(bar_q_full, (uint32_t)(q_tiles * C::kTileBytes));
-            for (int t = 0; t < kTilesPerCta; ++t) {
-                if (n_tiles[t] == 0) continue;
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(q_tile(t) + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64,
-                                m0 + t * kBlockM, h, b, pol_q);
-            }
+            mbar_arrive_expect_tx(bar_q_full, (uint32_t)C::kTileBytes);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, m0, h, b, pol_q);
+            int cnt = 0;
             int issued[C::kStages];
             for (int s = 0; s < C::kStages; ++s) issued[s] = -1;
-            bool ok = true;
+            auto load = [&](const CUtensorMap* m, int j) {
+                const int s = cnt % C::kStages;
+                const uint32_t round = (uint32_t)(cnt / C::kStages);
+                if (!wait_bounded(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, p.wait_limit)) return false;
+                mbar_arrive_expect_tx(bar_kv_full(s), (uint32_t)C::kTileBytes);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(kv_slot(s) + bx * kSwizzleBoxBytes, m, bar_kv_full(s), bx * 64, j * kBlockN, h,
+                                b, pol_kv);
+                issued[s] = cnt;
+                ++cnt;
+                return true;
+            };
+            bool ok = load(&tm_k, 0);
+            if (ok && n_kv > 1) ok = load(&tm_k, 1);
             for (int j = 0; j < n_kv && ok; ++j) {
-                for (int which = 0; which < 2 && ok; ++which) {
-                    const int n = 2 * j + which;
-                    const int s = n % C::kStages;
-                    const uint32_t round = (uint32_t)(n / C::kStages);
-                    if (!wait_bounded(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, p.wait_limit)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(bar_kv_full(s), (uint32_t)C::kTileBytes);
-                    const CUtensorMap* m = which == 0 ? &tm_k : &tm_v;
-                    for (int bx = 0; bx < C::kBoxes; ++bx)
-                        tma_load_4d(kv_slot(s) + bx * kSwizzleBoxBytes, m, bar_kv_full(s), bx * 64,
-                                    j * kBlockN, h, b, pol_kv);
-                    issued[s] = n;
-                }
+                ok = load(&tm_v, j);
+                if (ok && j + 2 < n_kv) ok = load(&tm_k, j + 2);
             }
             if (!ok) {
                 // wind down: let every copy already issued land before the CTA exits
@@ -267,103 +334,97 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         // =========================================================== MMA issuer
         if (lane == 0 && n_kv > 0) {
             bool ok = wait_bounded(bar_q_full, 0, abort_flag, p.wait_limit);
-            auto mma_qk = [&](int t, int slot) {
+            int cnt = 0;
+            auto next_slot = [&](int& s) {
+                s = cnt % C::kStages;
+                const bool r = wait_bounded(bar_kv_full(s), (uint32_t)((cnt / C::kStages) & 1), abort_flag,
+                                            p.wait_limit);
+                ++cnt;
+                return r;
+            };
+            auto mma_qk = [&](int buf, int slot) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
-                    const uint64_t a = smem_desc_sw128(q_tile(t) + koff, 16, 1024);
+                    const uint64_t a = smem_desc_sw128(q_tile + koff, 16, 1024);
                     const uint64_t bb = smem_desc_sw128(kv_slot(slot) + koff, 16, 1024);
-                    umma_ss(tmem + C::col_s(t), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + C::col_s(buf), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
                 }
             };
-            auto mma_pv = [&](int t, int slot, bool accumulate) {
+            auto mma_pv = [&](int buf, int slot, bool accumulate) {
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    // keys 16kk..16kk+15 of P: 8 bf16-pair columns per step
+                    const uint32_t a_col = C::col_s(buf) + (uint32_t)(kk * 8);
                     const uint64_t bb =
                         smem_desc_sw128(kv_slot(slot) + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024);
-                    umma_ts(tmem + C::col_o(t), tmem + C::col_p(t) + (uint32_t)(kk * 8), bb, C::kIdescPV,
-                            (accumulate || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
                 }
             };
-            auto kv_wait = [&](int n) {
-                const int s = n % C::kStages;
-                return wait_bounded(bar_kv_full(s), (uint32_t)((n / C::kStages) & 1), abort_flag, p.wait_limit);
-            };
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int sK = (2 * j) % C::kStages;
-                const int sV = (2 * j - 1 + 2 * C::kStages) % C::kStages;  // slot of V_{j-1}
-                ok = kv_wait(2 * j);
-                if (ok && j > 0) ok = kv_wait(2 * j - 1);
+            int s = 0;
+            for (int j = 0; j < 2 && j < n_kv && ok; ++j) {
+                ok = next_slot(s);
                 if (!ok) break;
                 tc_fence_after();
-                for (int t = 0; t < kTilesPerCta && ok; ++t) {
-                    if (j < n_tiles[t]) {
-                        if (j > 0) {
-                            ok = wait_bounded(bar_p_full(t), (uint32_t)((j - 1) & 1), abort_flag, p.wait_limit);
-                            if (!ok) break;
-                            tc_fence_after();
-                            mma_pv(t, sV, j - 1 > 0);
-                        }
-                        mma_qk(t, sK);
-                        umma_commit(bar_s_full(t));
-                    } else if (j == n_tiles[t] && j > 0) {
-                        ok = wait_bounded(bar_p_full(t), (uint32_t)((j - 1) & 1), abort_flag, p.wait_limit);
-                        if (!ok) break;
-                        tc_fence_after();
-                        mma_pv(t, sV, j - 1 > 0);
-                        umma_commit(bar_o_full(t));
-                    }
-                }
-                if (!ok) break;
-                umma_commit(bar_kv_empty(sK));
-                if (j > 0) umma_commit(bar_kv_empty(sV));
+                mma_qk(j, s);
+                umma_commit(bar_s_full(j));
+                umma_commit(bar_kv_empty(s));
             }
-            if (ok) {
-                const int j = n_kv;
-                const int sV = (2 * j - 1) % C::kStages;
-                ok = kv_wait(2 * j - 1);
-                if (ok) tc_fence_after();
-                for (int t = 0; t < kTilesPerCta && ok; ++t) {
-                    if (n_tiles[t] != n_kv) continue;
-                    ok = wait_bounded(bar_p_full(t), (uint32_t)((j - 1) & 1), abort_flag, p.wait_limit);
+            for (int j = 0; j < n_kv && ok; ++j) {
+                ok = next_slot(s);  // V_j
+                if (ok) ok = wait_bounded(bar_p_full(j & 1), (uint32_t)((j >> 1) & 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                tc_fence_after();
+                mma_pv(j & 1, s, j > 0);
+                umma_commit(bar_o_done(j & 1));
+                umma_commit(bar_kv_empty(s));
+                if (j + 2 < n_kv) {
+                    ok = next_slot(s);  // K_{j+2}
                     if (!ok) break;
                     tc_fence_after();
-                    mma_pv(t, sV, j - 1 > 0);
-                    umma_commit(bar_o_full(t));
+                    // overwrites S(j) and P(j): issued after the PV that reads P(j)
+                    mma_qk(j & 1, s);
+                    umma_commit(bar_s_full(j & 1));
+                    umma_commit(bar_kv_empty(s));
                 }
-                if (ok) umma_commit(bar_kv_empty(sV));
             }
             // drain: every MMA and commit of this CTA has landed before TMEM is freed
             umma_commit(bar_drain);
             (void)wait_bounded(bar_drain, 0, abort_flag, p.wait_limit);
         }
         __syncwarp();
+      }
     } else {
-        // =========================================================== softmax, one row per thread
-        const int t = warp >> 2;                       // Q tile of this warpgroup
-        const int r = threadIdx.x & (kBlockM - 1);     // row inside the tile == TMEM lane
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int row = m0 + t * kBlockM + r;
-        const int nt = n_tiles[t];
-        const bool tile_has_rows = (m0 + t * kBlockM) < p.Nq;
+        setmaxnreg_inc<kRegsSoftmax>();   // warpgroups 0 and 1
+        // =========================================================== softmax: one thread per row, alternate tiles
+        const int qd = warp & 3;                     // TMEM lane quadrant
+        const int par = warp >> 2;                   // this warp takes the tiles j with j % 2 == par
+        const int r = qd * 32 + lane;                // row inside the tile == TMEM lane
+        const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+        const int row = m0 + r;
         const int lim = row_key_limit(row, kl, off, p.causal);
         const float c = p.scale_log2;
-        float m_ref = -INFINITY;   // reference max (log2 units) shared by l and O
-        float l = 0.f;
+        float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
+        float l = 0.f;             // sum of this warp's probabilities, relative to m_seen
         bool ok = true;
 
-        for (int j = 0; j < nt; ++j) {
-            if (!wait_bounded(bar_s_full(t), (uint32_t)(j & 1), abort_flag, p.wait_limit)) {
+        for (int j = par; j < n_kv; j += 2) {
+            const int buf = j & 1;
+            bool good = wait_bounded(bar_s_full(buf), (uint32_t)((j >> 1) & 1), abort_flag, p.wait_limit);
+            if (!__all_sync(0xffffffffu, good)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            const int kbase = j * kBlockN;
+            // warp-uniform: the element mask runs only on tiles that cross a row's key limit
+            const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim);
             float s[kBlockN];
             {
                 uint32_t u[kBlockN];
 #pragma unroll
-                for (int q4 = 0; q4 < kBlockN / 32; ++q4)
-                    tmem_ld32(tmem + lane_off + C::col_s(t) + 32u * q4,
+                for (int q4 = 0; q4 < 4; ++q4)
+                    tmem_ld32(tmem + lane_off + C::col_s(buf) + 32u * q4,
                               *reinterpret_cast<uint32_t(*)[32]>(&u[32 * q4]));
                 tmem_wait_ld();
 #pragma unroll
@@ -372,122 +433,147 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     s[i] = __uint_as_float(u[i]);
                 }
             }
-            const int kbase = j * kBlockN;
-            if (kbase + kBlockN > lim) {
+            if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBlockN; ++i)
                     if (kbase + i >= lim) s[i] = -INFINITY;
             }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int i = 4; i < kBlockN; i += 4) {
-                mx0 = fmaxf(mx0, s[i]);
-                mx1 = fmaxf(mx1, s[i + 1]);
-                mx2 = fmaxf(mx2, s[i + 2]);
-                mx3 = fmaxf(mx3, s[i + 3]);
-            }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            const float t_max = mx * c;   // c > 0, so -inf stays -inf
-            const float m_new = fmaxf(m_ref, t_max);
-            float alpha = 1.f;
-            if (m_new > m_ref + kRescaleThreshold) {
-                alpha = ex2_approx(m_ref - m_new);  // 0 when m_ref is -inf
-                l *= alpha;
-                m_ref = m_new;
-            }
-            const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-            float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                // 64 probabilities -> 32 packed bf16 pairs -> TMEM columns of P
-                uint32_t w[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float e0 = ex2_approx(fmaf(s[64 * h2 + 2 * i], c, -mu));
-                    const float e1 = ex2_approx(fmaf(s[64 * h2 + 2 * i + 1], c, -mu));
-                    l0 += e0;
-                    l1 += e1;
-                    w[i] = pack_bf16x2(e0, e1);
+            const float mx = fmaxf(fmaxf(chunk_max32(s, 0), chunk_max32(s, 32)),
+                                   fmaxf(chunk_max32(s, 64), chunk_max32(s, 96)));
+            // reference max after tile j-1, published by the partner warp
+            float m_prev = -INFINITY;
+            if (j > 0) {
+                good = wait_bounded(bar_m_ready(qd, (j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
+                                    p.wait_limit);
+                if (!__all_sync(0xffffffffu, good)) {
+                    ok = false;
+                    break;
                 }
-                tmem_st32(tmem + lane_off + C::col_p(t) + 32u * h2, w);
+                m_prev = mref[((j - 1) & 1) * kBlockM + r];
             }
-            l += l0 + l1;
-            // O still holds the sum over tiles < j, relative to the old max.
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            const float t_max = mx * c;   // c > 0, so -inf stays -inf
+            const float m_cur = (t_max > m_prev + kRescaleThreshold) ? t_max : m_prev;
+            if (j + 1 < n_kv) {
+                mref[buf * kBlockM + r] = m_cur;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_m_ready(qd, buf));
+            }
+            if (m_cur != m_seen) {
+                l *= ex2_approx(m_seen - m_cur);  // 0 while m_seen is -inf
+                m_seen = m_cur;
+            }
+            const float mu = (m_cur == -INFINITY) ? 0.f : m_cur;
+            float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
+            const uint32_t taddr_p = tmem + lane_off + C::col_s(buf);
+            if (masked) {
+                exp_store_half<0, 0>(s, c, mu, taddr_p, l0, l1);
+                exp_store_half<0, 1>(s, c, mu, taddr_p, l0, l1);
+            } else {
+                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, l0, l1);
+                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, l0, l1);
+            }
+            l += (l0.x + l0.y) + (l1.x + l1.y);
+            if (j > 0) {
+                // O holds tiles < j relative to m_prev once the PV of tile j-1 is done
+                good = wait_bounded(bar_o_done((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
+                                    p.wait_limit);
+                if (!__all_sync(0xffffffffu, good)) {
+                    tmem_wait_st();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float alpha = (m_cur != m_prev) ? ex2_approx(m_prev - m_cur) : 1.f;
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                for (int q4 = 0; q4 < D / 32; ++q4) {
-                    uint32_t u[32];
-                    tmem_ld32(tmem + lane_off + C::col_o(t) + 32u * q4, u);
-                    tmem_wait_ld();
+                    for (int q4 = 0; q4 < D / 32; ++q4) {
+                        const uint32_t ocol = tmem + lane_off + C::kColO + 32u * q4;
+                        uint32_t u[32];
+                        tmem_ld32(ocol, u);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        reg_after_wait(u[i]);
-                        u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        for (int i = 0; i < 32; i += 2) {
+                            reg_after_wait(u[i]);
+                            reg_after_wait(u[i + 1]);
+                            const float2 v = __fmul2_rn(
+                                make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                make_float2(alpha, alpha));
+                            u[i] = __float_as_uint(v.x);
+                            u[i + 1] = __float_as_uint(v.y);
+                        }
+                        tmem_st32(ocol, u);
                     }
-                    tmem_st32(tmem + lane_off + C::col_o(t) + 32u * q4, u);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p_full(t));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p_full(buf));
         }
 
         // ---------------------------------------------------------- epilogue
-        if (ok && tile_has_rows) {
-            bool have_o = nt > 0;
-            if (have_o) {
-                if (!wait_bounded(bar_o_full(t), 0, abort_flag, p.wait_limit)) {
-                    ok = false;
-                    have_o = false;
+        // Exits and skipped stores are decided jointly (bar.red.or), so a wait
+        // that ran out never leaves another warp stuck at a named barrier.
+        const bool have_o = n_kv > 0;
+        bool good = ok;
+        if (good && have_o) {
+            good = wait_bounded(bar_o_done((n_kv - 1) & 1), (uint32_t)(((n_kv - 1) >> 1) & 1), abort_flag,
+                                p.wait_limit);
+            good = __all_sync(0xffffffffu, good);
+            if (good) tc_fence_after();
+        }
+        epi[par * kBlockM + r] = m_seen;
+        epi[(2 + par) * kBlockM + r] = l;
+        good = !named_bar_or(kBarQuadBase + qd, 64, !good);
+        // both warps' sums, brought to the final (largest) reference max
+        const float m_oth = epi[(par ^ 1) * kBlockM + r];
+        const float l_oth = epi[(2 + (par ^ 1)) * kBlockM + r];
+        const float m_fin = fmaxf(m_seen, m_oth);
+        const float l_row = (m_seen == m_fin ? l : l * ex2_approx(m_seen - m_fin)) +
+                            (m_oth == m_fin ? l_oth : l_oth * ex2_approx(m_oth - m_fin));
+        if (good) {
+            const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
+#pragma unroll
+            for (int q4 = 0; q4 < D / 64; ++q4) {
+                const int col0 = par * (D / 2) + 32 * q4;   // first O column of this chunk
+                uint32_t u[32];
+                if (have_o) {
+                    tmem_ld32(tmem + lane_off + C::kColO + (uint32_t)col0, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) reg_after_wait(u[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) u[i] = 0u;
                 }
-                tc_fence_after();
-            }
-            if (ok) {
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                const uint32_t stage = q_tile(t);
+                uint32_t pkd[16];
 #pragma unroll
-                for (int q4 = 0; q4 < D / 32; ++q4) {
-                    uint32_t u[32];
-                    if (have_o) {
-                        tmem_ld32(tmem + lane_off + C::col_o(t) + 32u * q4, u);
-                        tmem_wait_ld();
+                for (int i = 0; i < 16; ++i)
+                    pkd[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+                // 4 x 16-byte chunks of row r; chunk cc of the row lives in box cc/8,
+                // swizzled position (cc%8) ^ (r%8) inside the row's 128 bytes.
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) reg_after_wait(u[i]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) u[i] = 0u;
-                    }
-                    uint32_t pkd[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pkd[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l,
-                                             __uint_as_float(u[2 * i + 1]) * inv_l);
-                    // 4 x 16-byte chunks of row r; chunk cc of the row lives in box cc/8,
-                    // swizzled position (cc%8) ^ (r%8) inside the row's 128 bytes.
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        const int cc = q4 * 4 + v4;
-                        const uint32_t addr = stage + (uint32_t)((cc >> 3) * kSwizzleBoxBytes + r * 128 +
-                                                                 (((cc & 7) ^ (r & 7)) << 4));
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                     "r"(pkd[4 * v4]), "r"(pkd[4 * v4 + 1]), "r"(pkd[4 * v4 + 2]),
-                                     "r"(pkd[4 * v4 + 3])
-                                     : "memory");
-                    }
-                }
-                if (row < p.Nq) {
-                    const float lse = (l > 0.f) ? (m_ref + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
-                    p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
-                }
-                fence_proxy_async_smem();
-                named_bar_sync(1 + t, kBlockM);
-                if (r == 0) {
-                    for (int bx = 0; bx < C::kBoxes; ++bx)
-                        tma_store_4d(&tm_o, stage + bx * kSwizzleBoxBytes, bx * 64, m0 + t * kBlockM, h, b);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    const int cc = col0 / 8 + v4;
+                    const uint32_t addr = q_tile + (uint32_t)((cc >> 3) * kSwizzleBoxBytes + r * 128 +
+                                                              (((cc & 7) ^ (r & 7)) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pkd[4 * v4]),
+                                 "r"(pkd[4 * v4 + 1]), "r"(pkd[4 * v4 + 2]), "r"(pkd[4 * v4 + 3])
+                                 : "memory");
                 }
             }
+            if (par == 0 && row < p.Nq) {
+                const float lse = (l_row > 0.f) ? (m_fin + lg2_approx(l_row)) * 0.69314718055994531f : -INFINITY;
+                p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
+            }
+        }
+        fence_proxy_async_smem();
+        const bool any_bad = named_bar_or(kBarSoftmaxAll, kSoftmaxWarps * 32, !good);
+        if (!any_bad && threadIdx.x == 0) {
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_store_4d(&tm_o, q_tile + bx * kSwizzleBoxBytes, bx * 64, m0, h, b);
+            bulk_commit_group();
+            bulk_wait_group_read0();
         }
         tc_fence_before();
     }
