@@ -227,6 +227,21 @@ def oracle_sample_rate(w, x, target_s, rng_seed=0):
     return n * flop_per_row / t / 1e12, n, t, oracle.num_threads()
 
 
+def job_time_ms(local_ms: float, world: int, device="cpu") -> float:
+    """Job time = the slowest rank's timed region (max over ranks; no data moves)."""
+    if world <= 1:
+        return float(local_ms)
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_tflops(flop_per_step: float, steps: int, world: int, job_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica of the workload."""
+    return world * steps * flop_per_step / (job_ms / 1000.0) / 1e12
+
+
 def config_of(w, l2_note, parallelism):
     mask = "causal" if w.causal else "none"
     if w.key_len_range:
@@ -306,11 +321,8 @@ def main():
     status = fa_get_device_status()
     if status != FA_OK:
         raise SystemExit(f"device status {status} after the timed region")
-    t_total = torch.tensor([sum(per)], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t_total, op=torch.distributed.ReduceOp.MAX)
-    job_ms = float(t_total.item())
-    value = world * args.steps * w.flop / (job_ms / 1000.0) / 1e12
+    job_ms = job_time_ms(sum(per), world, device)
+    value = job_throughput_tflops(w.flop, args.steps, world, job_ms)
 
     peaks, peaks_src = load_peaks()
     peak = float(peaks["bf16_tflops"])

@@ -9,23 +9,31 @@
 // Hopper; this one is laid out for Blackwell:
 //
 //  * one CTA = one (b, h) and one 128-row Q tile (TMEM lane i = query row i);
-//  * warp 8 (one elected lane) loads Q once and then streams K and V tiles
-//    (128 keys) through a ring of shared-memory slots with TMA (128B-swizzled
-//    boxes of 64 columns x 128 rows), one full/empty mbarrier pair per slot --
-//    the double buffering "FlashAttention：把注意力从公式写成数据流" (section
-//    "端侧与专用加速器") names for hiding loads;
-//  * warp 9 (one elected lane) issues the tcgen05 MMAs.  S is double-buffered
-//    in TMEM: S(j+2) = Q K_{j+2}^T is issued right after O += P(j) V_j, so the
-//    score tile the softmax needs next is computed while it works on the
-//    current one and the softmax never waits on the tensor core;
-//  * warps 0-7 do the online softmax, one thread per query row and tile:
-//    warps q and q+4 both own TMEM lanes 32q..32q+31 and take the K/V tiles
-//    in turn (even / odd), so one warp's exponentials overlap the other's
-//    loads and maxima.  Only the running reference max passes between them
-//    (shared memory + an mbarrier); each keeps its own partial row sum.
-//    Exponentials are taken in the exp2 domain, some on MUFU and some with a
-//    polynomial on the FMA pipe; P goes back to TMEM as bf16 over the first
-//    half of the tile's S buffer and feeds the PV MMA from there;
+//  * warp 8 (one elected lane) loads Q once and then streams the K tiles (128
+//    keys), warp 10 the V tiles, each through its own ring of shared-memory
+//    slots with TMA (128B-swizzled boxes of 64 columns x 128 rows), one
+//    full/empty mbarrier pair per slot -- the double buffering
+//    "FlashAttention：把注意力从公式写成数据流" (section "端侧与专用加速器") names
+//    for hiding loads;
+//  * two warps (one elected lane each) issue the tcgen05 MMAs: warp 9 the
+//    S(i) = Q K_i^T products into the TMEM score buffer(s), warp 11 the
+//    O += P(j) V_j products.  The two streams touch disjoint TMEM and
+//    separate rings, so neither waits for the other and the tensor core is
+//    fed by one while the other waits on a barrier;
+//  * P is written to its own TMEM buffers (three, 64 columns of bf16 pairs
+//    each), never over the scores: a PV product followed by a QK^T product
+//    into the columns it has just read is a write-after-read on TMEM that the
+//    tensor core resolves by draining.  Scores are read out within a few
+//    hundred cycles of landing, so one score buffer (two at d = 64, where
+//    TMEM has room) keeps the QK^T stream going;
+//  * warps 0-7 do the online softmax, one thread per query row: warps q and
+//    q+4 both own TMEM lanes 32q..32q+31 and take the K/V tiles in turn (even
+//    / odd), each holding a whole 128-key row in registers.  A score buffer
+//    is handed back as soon as it has been read, so the next QK^T product
+//    overlaps the exponentials.  Only the running reference max passes
+//    between the two warps (shared memory + an mbarrier); each keeps its own
+//    partial row sums.  Exponentials are taken in the exp2 domain, some on
+//    MUFU and some with a polynomial on the FMA pipe;
 //  * the reference max moves only when the row max grows by more than 2^8;
 //    O is then rescaled in TMEM (exact: m, l and O always share one max);
 //  * epilogue: O / l -> bf16 -> shared memory (128B-swizzled) -> TMA store
@@ -50,20 +58,23 @@ namespace fa {
 
 constexpr int kBlockM = 128;        // query rows per CTA (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
-constexpr int kNumThreads = 384;    // 8 softmax warps, producer, MMA, 2 spare
-constexpr int kSoftmaxWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kGroups = 2;          // softmax warps per TMEM lane quadrant (tiles taken in turn)
+constexpr int kSoftmaxWarps = 4 * kGroups;
+constexpr int kNumThreads = 384;    // 8 softmax warps, 2 TMA producers, 2 MMA issuers
+constexpr int kProducerWarp = 8;    // Q and the K tiles
+constexpr int kMmaWarp = 9;         // issues the QK^T products (and owns the TMEM allocation)
+constexpr int kVProducerWarp = 10;  // the V tiles
+constexpr int kPvWarp = 11;         // issues the PV products
 constexpr int kTmemCols = 512;
 // Registers are allocated per warpgroup: 384 threads x 168 at launch, then the
-// softmax warpgroups take 216 and the producer/MMA warpgroup keeps 72
-// (2*128*216 + 128*72 = 384*168).
-constexpr uint32_t kRegsSoftmax = 216;
-constexpr uint32_t kRegsControl = 72;
+// two softmax warpgroups take 200 and the producer/MMA warpgroup keeps 104
+// (2*128*200 + 128*104 <= 384*168).
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsControl = 104;
 constexpr int kSwizzleBoxBytes = 128 * 128;  // one 64-column x 128-row bf16 box
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only if max grows > 2^8
 constexpr int kStatusTimeout = -6;           // FA_ERR_DEVICE_TIMEOUT
-// named barriers (epilogue only): 1..4 pair the two warps of a lane quadrant, 5 spans all softmax warps
+// named barriers (epilogue only): 1..4 join the warps of a lane quadrant, 5 spans all softmax warps
 constexpr uint32_t kBarQuadBase = 1;
 constexpr uint32_t kBarSoftmaxAll = 5;
 
@@ -81,28 +92,39 @@ struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kBoxes = D / 64;                        // 64-column boxes per row
     static constexpr int kTileBytes = kBlockM * D * 2;           // one Q / K / V tile
-    static constexpr int kStages = (D == 64) ? 10 : 5;           // K/V ring slots
+    static constexpr int kStagesK = (D == 64) ? 6 : 3;           // K ring slots
+    static constexpr int kStagesV = (D == 64) ? 6 : 2;           // V ring slots
+    static constexpr int kStages = kStagesK + kStagesV;
     // Of every 8 pairs of probabilities, this many are computed on the FMA pipe
     // (exp2_fma2) and the rest on MUFU, so neither unit is the lone bottleneck.
 #ifdef FA_EMU_PAIRS_D64
     static constexpr int kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
 #else
-    static constexpr int kEmuPairs = 2;
+    static constexpr int kEmuPairs = 1;
 #endif
     static constexpr int kQOff = 0;
-    static constexpr int kKvOff = kTileBytes;
-    static constexpr int kBarOff = kKvOff + kStages * kTileBytes;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
-    // m_ready[4 quadrants][2 parities], drain
-    static constexpr int kNumBars = 16 + 2 * kStages;
+    static constexpr int kKOff = kTileBytes;
+    static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
+    static constexpr int kBarOff = kVOff + kStagesV * kTileBytes;
+    static constexpr int kSBufs = (D == 64) ? 2 : 1;             // TMEM score buffers
+    static constexpr int kPBufs = 3;                             // TMEM probability buffers
+    // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
+    // s_full[2 (per softmax warp)], s_free[2], p_full[3], pv_done[3],
+    // m_ready[4 quadrants][2], drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 3 + 3 + 8 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
-    static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [parity][row]
-    static constexpr int kEpiOff = kMrefOff + 2 * kBlockM * 4;   // epilogue exchange: m [2][row], l [2][row]
-    static constexpr int kSmemBytes = kEpiOff + 4 * kBlockM * 4 + 1024;  // + alignment slack
-    // TMEM columns: S buffers at 0 and 128 (P of a tile over the first 64
-    // columns of its S buffer), O at 256.
+    static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row]
+    static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, l, lu [2][row] each
+    static constexpr int kSmemBytes = kEpiOff + 3 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
+    static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
+    // TMEM columns: S buffers from 0 (128 each), then the P buffers (bf16
+    // pairs, 64 each), O in the last D columns.
+    //   D = 128: S 0..127, P 128..319, O 384..511
+    //   D = 64:  S 0..255, P 256..447, O 448..511
     __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
-    static constexpr uint32_t kColO = 256;
+    __host__ __device__ static constexpr uint32_t col_p(int b) { return 128u * kSBufs + 64u * b; }
+    static constexpr uint32_t kColO = 512u - D;
+    static_assert(128 * kSBufs + 64 * kPBufs <= 512 - D, "TMEM columns");
     // Instruction descriptors (kind::f16): D=f32, A=B=bf16, M=128.
     //   QK^T: A=Q K-major, B=K K-major, N=128.  PV: A=P (TMEM, K-major), B=V MN-major, N=D.
     static constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
@@ -134,9 +156,9 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        // sleeps until the phase completes (or 0.1 ms passes): a waiting warp
-        // leaves its issue slots to the warps that are computing
-        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        // plain try_wait: an explicit suspend-time hint wakes the waiter
+        // noticeably later after the phase completes
+        if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
         if ((unsigned long long)(clock64() - t0) > limit) {
             *abort_flag = 1;
@@ -165,12 +187,14 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 // p = 2^(s*c - mu) for keys 64*h2 .. 64*h2+63 of the thread's row, packed to
-// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2; the fp32 p are
-// summed into (l0, l1).  kEmu of every 8 pairs go through exp2_fma2, the rest
-// through MUFU ex2 (which maps -inf to 0, so masked tiles use kEmu = 0).
+// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2.  Two row sums: lr
+// adds the bf16-rounded p (the weights the PV product uses, so O is normalised
+// consistently), lu the unrounded p (for the log-sum-exp).  kEmu of every 8
+// pairs go through exp2_fma2, the rest through MUFU ex2 (which maps -inf to 0,
+// so masked tiles use kEmu = 0).
 template <int kEmu, int h2>
 __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float c, float mu, uint32_t taddr_p,
-                                               float2& l0, float2& l1) {
+                                               float2& lr, float2& lu) {
     const float2 c2 = make_float2(c, c);
     const float2 nmu = make_float2(-mu, -mu);
     uint32_t w[32];
@@ -185,11 +209,9 @@ __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float 
             e.x = ex2_approx(x.x);
             e.y = ex2_approx(x.y);
         }
-        if (i & 1)
-            l1 = __fadd2_rn(l1, e);
-        else
-            l0 = __fadd2_rn(l0, e);
         w[i] = pack_bf16x2(e.x, e.y);
+        lu = __fadd2_rn(lu, e);
+        lr = __fadd2_rn(lr, make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)));
     }
     tmem_st32(taddr_p + 32u * h2, w);
 }
@@ -224,19 +246,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint8_t* const base_ptr = smem_raw + (base - raw_base);
 
     const uint32_t bar_q_full = base + C::kBarOff;
-    auto bar_kv_full = [&](int s) { return base + C::kBarOff + 8u * (1 + s); };
-    auto bar_kv_empty = [&](int s) { return base + C::kBarOff + 8u * (1 + C::kStages + s); };
-    auto bar_s_full = [&](int b) { return base + C::kBarOff + 8u * (1 + 2 * C::kStages + b); };
-    auto bar_p_full = [&](int b) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + b); };
-    auto bar_o_done = [&](int b) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + b); };
-    auto bar_m_ready = [&](int qd, int b) { return base + C::kBarOff + 8u * (7 + 2 * C::kStages + 2 * qd + b); };
-    const uint32_t bar_drain = base + C::kBarOff + 8u * (15 + 2 * C::kStages);
+    // ring r = 0 (K, kStagesK slots) or 1 (V, kStagesV slots): full barriers
+    // of both rings, then the empty ones
+    auto bar_full = [&](int r, int s) { return base + C::kBarOff + 8u * (1 + r * C::kStagesK + s); };
+    auto bar_empty = [&](int r, int s) { return base + C::kBarOff + 8u * (1 + C::kStages + r * C::kStagesK + s); };
+    auto bar_s_full = [&](int g) { return base + C::kBarOff + 8u * (1 + 2 * C::kStages + g); };
+    auto bar_s_free = [&](int b) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + b); };
+    auto bar_p_full = [&](int b) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + b); };
+    auto bar_pv_done = [&](int b) { return base + C::kBarOff + 8u * (8 + 2 * C::kStages + b); };
+    auto bar_m_ready = [&](int qd, int g) { return base + C::kBarOff + 8u * (11 + 2 * C::kStages + 2 * qd + g); };
+    const uint32_t bar_drain = base + C::kBarOff + 8u * (19 + 2 * C::kStages);
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
-    float* const mref = reinterpret_cast<float*>(base_ptr + C::kMrefOff);     // [parity][row]
-    float* const epi = reinterpret_cast<float*>(base_ptr + C::kEpiOff);       // m [2][row], l [2][row]
+    float* const mref = reinterpret_cast<float*>(base_ptr + C::kMrefOff);     // [group][row]
+    float* const epi = reinterpret_cast<float*>(base_ptr + C::kEpiOff);       // m, l, lu [group][row] each
     const uint32_t q_tile = base + C::kQOff;
-    auto kv_slot = [&](int s) { return base + C::kKvOff + (uint32_t)(s * C::kTileBytes); };
+    auto ring_slot = [&](int r, int s) {
+        return base + (r == 0 ? C::kKOff : C::kVOff) + (uint32_t)(s * C::kTileBytes);
+    };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -260,18 +287,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ---- setup: barriers (producer lane 0), TMEM (MMA warp)
     if (warp == kProducerWarp && lane == 0) {
         mbar_init(bar_q_full, 1);
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(bar_kv_full(s), 1);
-            mbar_init(bar_kv_empty(s), 1);
+        for (int r2 = 0; r2 < 2; ++r2)
+            for (int s = 0; s < (r2 == 0 ? C::kStagesK : C::kStagesV); ++s) {
+                mbar_init(bar_full(r2, s), 1);
+                mbar_init(bar_empty(r2, s), 1);
+            }
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(bar_s_full(g), 1);
+            mbar_init(bar_s_free(g), 4);    // one arrival per lane quadrant
         }
-        mbar_init(bar_s_full(0), 1);
-        mbar_init(bar_s_full(1), 1);
-        for (int b2 = 0; b2 < 2; ++b2) {
-            mbar_init(bar_p_full(b2), kSoftmaxWarps / 2);
-            mbar_init(bar_o_done(b2), 1);
+        for (int b2 = 0; b2 < C::kPBufs; ++b2) {
+            mbar_init(bar_p_full(b2), 4);   // one arrival per lane quadrant
+            mbar_init(bar_pv_done(b2), 1);
         }
         for (int i = 0; i < 8; ++i) mbar_init(bar_m_ready(i >> 1, i & 1), 1);
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain, 2);   // one commit from each MMA issuer
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_q);
@@ -288,107 +318,96 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    // The K/V load order, shared by producer and MMA issuer: K0, K1, then for
-    // every j: V_j followed by K_{j+2} -- the order the MMAs consume them in.
     if (warp >= kProducerWarp) {
       setmaxnreg_dec<kRegsControl>();   // whole warpgroup 2, one instruction
-      if (warp == kProducerWarp) {
-        // =========================================================== TMA producer
+      if (warp == kProducerWarp || warp == kVProducerWarp) {
+        // =========================================================== TMA producers
+        // Each streams its own tensor, tiles 0 .. n_kv-1 in order, through its
+        // own ring; warp 8 also loads the Q tile first.
+        const int rg = (warp == kProducerWarp) ? 0 : 1;
+        const CUtensorMap* const tm = (rg == 0) ? &tm_k : &tm_v;
+        const int ns = (rg == 0) ? C::kStagesK : C::kStagesV;
         if (lane == 0 && n_kv > 0) {
             const uint64_t pol_kv = policy_evict_last();
-            const uint64_t pol_q = policy_evict_first();
-            mbar_arrive_expect_tx(bar_q_full, (uint32_t)C::kTileBytes);
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-                tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, m0, h, b, pol_q);
-            int cnt = 0;
-            int issued[C::kStages];
-            for (int s = 0; s < C::kStages; ++s) issued[s] = -1;
-            auto load = [&](const CUtensorMap* m, int j) {
-                const int s = cnt % C::kStages;
-                const uint32_t round = (uint32_t)(cnt / C::kStages);
-                if (!wait_bounded(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, p.wait_limit)) return false;
-                mbar_arrive_expect_tx(bar_kv_full(s), (uint32_t)C::kTileBytes);
+            if (rg == 0) {
+                mbar_arrive_expect_tx(bar_q_full, (uint32_t)C::kTileBytes);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(kv_slot(s) + bx * kSwizzleBoxBytes, m, bar_kv_full(s), bx * 64, j * kBlockN, h,
-                                b, pol_kv);
-                issued[s] = cnt;
-                ++cnt;
-                return true;
-            };
-            bool ok = load(&tm_k, 0);
-            if (ok && n_kv > 1) ok = load(&tm_k, 1);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                ok = load(&tm_v, j);
-                if (ok && j + 2 < n_kv) ok = load(&tm_k, j + 2);
+                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, m0, h, b,
+                                policy_evict_first());
+            }
+            bool ok = true;
+            int j = 0;
+            for (; j < n_kv && ok; ++j) {
+                const int s = j % ns;
+                const uint32_t round = (uint32_t)(j / ns);
+                ok = wait_bounded(bar_empty(rg, s), (round & 1u) ^ 1u, abort_flag, p.wait_limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_full(rg, s), (uint32_t)C::kTileBytes);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64, j * kBlockN,
+                                h, b, pol_kv);
             }
             if (!ok) {
-                // wind down: let every copy already issued land before the CTA exits
-                for (int s = 0; s < C::kStages; ++s)
-                    if (issued[s] >= 0)
-                        (void)wait_bounded(bar_kv_full(s), (uint32_t)((issued[s] / C::kStages) & 1), abort_flag,
-                                           p.wait_limit);
+                // wind down: let every copy still in flight (at most one per
+                // slot, the newest ones) land before the CTA exits
+                for (int c2 = (j > ns ? j - ns : 0); c2 < j; ++c2)
+                    (void)wait_bounded(bar_full(rg, c2 % ns), (uint32_t)((c2 / ns) & 1), abort_flag, p.wait_limit);
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // =========================================================== MMA issuer
+    } else {
+        // =========================================================== MMA issuers
         if (lane == 0 && n_kv > 0) {
-            bool ok = wait_bounded(bar_q_full, 0, abort_flag, p.wait_limit);
-            int cnt = 0;
-            auto next_slot = [&](int& s) {
-                s = cnt % C::kStages;
-                const bool r = wait_bounded(bar_kv_full(s), (uint32_t)((cnt / C::kStages) & 1), abort_flag,
-                                            p.wait_limit);
-                ++cnt;
-                return r;
-            };
-            auto mma_qk = [&](int buf, int slot) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
-                    const uint64_t a = smem_desc_sw128(q_tile + koff, 16, 1024);
-                    const uint64_t bb = smem_desc_sw128(kv_slot(slot) + koff, 16, 1024);
-                    umma_ss(tmem + C::col_s(buf), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto mma_pv = [&](int buf, int slot, bool accumulate) {
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    // keys 16kk..16kk+15 of P: 8 bf16-pair columns per step
-                    const uint32_t a_col = C::col_s(buf) + (uint32_t)(kk * 8);
-                    const uint64_t bb =
-                        smem_desc_sw128(kv_slot(slot) + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024);
-                    umma_ts(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
-                }
-            };
-            int s = 0;
-            for (int j = 0; j < 2 && j < n_kv && ok; ++j) {
-                ok = next_slot(s);
-                if (!ok) break;
-                tc_fence_after();
-                mma_qk(j, s);
-                umma_commit(bar_s_full(j));
-                umma_commit(bar_kv_empty(s));
-            }
-            for (int j = 0; j < n_kv && ok; ++j) {
-                ok = next_slot(s);  // V_j
-                if (ok) ok = wait_bounded(bar_p_full(j & 1), (uint32_t)((j >> 1) & 1), abort_flag, p.wait_limit);
-                if (!ok) break;
-                tc_fence_after();
-                mma_pv(j & 1, s, j > 0);
-                umma_commit(bar_o_done(j & 1));
-                umma_commit(bar_kv_empty(s));
-                if (j + 2 < n_kv) {
-                    ok = next_slot(s);  // K_{j+2}
+            bool ok = true;
+            if (warp == kMmaWarp) {
+                ok = wait_bounded(bar_q_full, 0, abort_flag, p.wait_limit);
+                for (int i = 0; i < n_kv && ok; ++i) {
+                    // S(i - kSBufs) has been read into registers (first tiles: free buffer)
+                    const int t = i - C::kSBufs;
+                    if (t >= 0)
+                        ok = wait_bounded(bar_s_free(t % C::kSBufs), (uint32_t)((t / C::kSBufs) & 1), abort_flag,
+                                          p.wait_limit);
+                    const int sl = i % C::kStagesK;
+                    if (ok) ok = wait_bounded(bar_full(0, sl), (uint32_t)((i / C::kStagesK) & 1), abort_flag,
+                                              p.wait_limit);
                     if (!ok) break;
                     tc_fence_after();
-                    // overwrites S(j) and P(j): issued after the PV that reads P(j)
-                    mma_qk(j & 1, s);
-                    umma_commit(bar_s_full(j & 1));
-                    umma_commit(bar_kv_empty(s));
+                    const uint32_t slot = ring_slot(0, sl);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
+                        const uint64_t a = smem_desc_sw128(q_tile + koff, 16, 1024);
+                        const uint64_t bb = smem_desc_sw128(slot + koff, 16, 1024);
+                        umma_ss(tmem + C::col_s(i % C::kSBufs), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_s_full(i & 1));   // per softmax warp: tiles i, i+2, ...
+                    umma_commit(bar_empty(0, sl));
+                }
+            } else {
+                for (int j = 0; j < n_kv && ok; ++j) {
+                    // P(j) is in TMEM, and V_j has landed
+                    const int pb = j % C::kPBufs;
+                    ok = wait_bounded(bar_p_full(pb), (uint32_t)((j / C::kPBufs) & 1), abort_flag, p.wait_limit);
+                    const int sl = j % C::kStagesV;
+                    if (ok) ok = wait_bounded(bar_full(1, sl), (uint32_t)((j / C::kStagesV) & 1), abort_flag,
+                                              p.wait_limit);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t slot = ring_slot(1, sl);
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                        // keys 16kk..16kk+15 of P: 8 bf16-pair columns per step
+                        const uint32_t a_col = C::col_p(pb) + (uint32_t)(kk * 8);
+                        const uint64_t bb =
+                            smem_desc_sw128(slot + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024);
+                        umma_ts(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_pv_done(pb));
+                    umma_commit(bar_empty(1, sl));
                 }
             }
-            // drain: every MMA and commit of this CTA has landed before TMEM is freed
+            // drain: every MMA and commit of this CTA has landed before TMEM is
+            // freed (the barrier completes once both issuers have committed)
             umma_commit(bar_drain);
             (void)wait_bounded(bar_drain, 0, abort_flag, p.wait_limit);
         }
@@ -396,35 +415,33 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();   // warpgroups 0 and 1
-        // =========================================================== softmax: one thread per row, alternate tiles
+        // =========================================================== softmax: one thread per row, tiles in turn
         const int qd = warp & 3;                     // TMEM lane quadrant
-        const int par = warp >> 2;                   // this warp takes the tiles j with j % 2 == par
+        const int g = warp >> 2;                     // this warp takes the tiles j with j % 2 == g
         const int r = qd * 32 + lane;                // row inside the tile == TMEM lane
         const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
         const int row = m0 + r;
         const int lim = row_key_limit(row, kl, off, p.causal);
         const float c = p.scale_log2;
         float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
-        float l = 0.f;             // sum of this warp's probabilities, relative to m_seen
+        float l = 0.f;             // this warp's rounded probabilities, relative to m_seen
+        float lu = 0.f;            // the same sum before rounding (for the LSE)
         bool ok = true;
 
-        for (int j = par; j < n_kv; j += 2) {
-            const int buf = j & 1;
-            bool good = wait_bounded(bar_s_full(buf), (uint32_t)((j >> 1) & 1), abort_flag, p.wait_limit);
+        for (int j = g; j < n_kv; j += 2) {
+            const uint32_t use = (uint32_t)((j >> 1) & 1);   // phase parity of this tile in buffers g
+            bool good = wait_bounded(bar_s_full(g), use, abort_flag, p.wait_limit);
             if (!__all_sync(0xffffffffu, good)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int kbase = j * kBlockN;
-            // warp-uniform: the element mask runs only on tiles that cross a row's key limit
-            const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim);
             float s[kBlockN];
             {
                 uint32_t u[kBlockN];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
-                    tmem_ld32(tmem + lane_off + C::col_s(buf) + 32u * q4,
+                    tmem_ld32(tmem + lane_off + C::col_s(j % C::kSBufs) + 32u * q4,
                               *reinterpret_cast<uint32_t(*)[32]>(&u[32 * q4]));
                 tmem_wait_ld();
 #pragma unroll
@@ -433,6 +450,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     s[i] = __uint_as_float(u[i]);
                 }
             }
+            // the score buffer is free for S(j + kSBufs)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s_free(j % C::kSBufs));
+            const int kbase = j * kBlockN;
+            // warp-uniform: the element mask runs only on tiles that cross a row's key limit
+            const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim);
             if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBlockN; ++i)
@@ -440,75 +464,88 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             }
             const float mx = fmaxf(fmaxf(chunk_max32(s, 0), chunk_max32(s, 32)),
                                    fmaxf(chunk_max32(s, 64), chunk_max32(s, 96)));
-            // reference max after tile j-1, published by the partner warp
+            // reference max after tile j-1, published by the other warp of the quadrant
             float m_prev = -INFINITY;
             if (j > 0) {
-                good = wait_bounded(bar_m_ready(qd, (j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
+                good = wait_bounded(bar_m_ready(qd, g ^ 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
                                     p.wait_limit);
                 if (!__all_sync(0xffffffffu, good)) {
                     ok = false;
                     break;
                 }
-                m_prev = mref[((j - 1) & 1) * kBlockM + r];
+                m_prev = mref[(g ^ 1) * kBlockM + r];
             }
             const float t_max = mx * c;   // c > 0, so -inf stays -inf
             const float m_cur = (t_max > m_prev + kRescaleThreshold) ? t_max : m_prev;
             if (j + 1 < n_kv) {
-                mref[buf * kBlockM + r] = m_cur;
+                mref[g * kBlockM + r] = m_cur;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_m_ready(qd, buf));
+                if (lane == 0) mbar_arrive(bar_m_ready(qd, g));
             }
             if (m_cur != m_seen) {
-                l *= ex2_approx(m_seen - m_cur);  // 0 while m_seen is -inf
+                const float f = ex2_approx(m_seen - m_cur);  // 0 while m_seen is -inf
+                l *= f;
+                lu *= f;
                 m_seen = m_cur;
             }
             const float mu = (m_cur == -INFINITY) ? 0.f : m_cur;
-            float2 l0 = make_float2(0.f, 0.f), l1 = make_float2(0.f, 0.f);
-            const uint32_t taddr_p = tmem + lane_off + C::col_s(buf);
-            if (masked) {
-                exp_store_half<0, 0>(s, c, mu, taddr_p, l0, l1);
-                exp_store_half<0, 1>(s, c, mu, taddr_p, l0, l1);
-            } else {
-                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, l0, l1);
-                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, l0, l1);
-            }
-            l += (l0.x + l0.y) + (l1.x + l1.y);
-            if (j > 0) {
-                // O holds tiles < j relative to m_prev once the PV of tile j-1 is done
-                good = wait_bounded(bar_o_done((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
+            // P buffer j % 3 was last read by PV(j-3)
+            const int pb = j % C::kPBufs;
+            if (j >= C::kPBufs) {
+                good = wait_bounded(bar_pv_done(pb), (uint32_t)(((j - C::kPBufs) / C::kPBufs) & 1), abort_flag,
                                     p.wait_limit);
+                if (!__all_sync(0xffffffffu, good)) {
+                    ok = false;
+                    break;
+                }
+            }
+            float2 lr2 = make_float2(0.f, 0.f), lu2 = make_float2(0.f, 0.f);
+            const uint32_t taddr_p = tmem + lane_off + C::col_p(pb);
+            if (masked) {
+                exp_store_half<0, 0>(s, c, mu, taddr_p, lr2, lu2);
+                exp_store_half<0, 1>(s, c, mu, taddr_p, lr2, lu2);
+            } else {
+                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, lr2, lu2);
+                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, lr2, lu2);
+            }
+            l += lr2.x + lr2.y;
+            lu += lu2.x + lu2.y;
+            // O holds tiles < j relative to m_prev.  Only when some row of this
+            // warp moved its reference max does O have to be rescaled, and only
+            // then must PV(j-1) be complete first; PV(j) waits for this warp's
+            // P-ready arrival, so it cannot have started.
+            const float alpha = (m_cur != m_prev) ? ex2_approx(m_prev - m_cur) : 1.f;
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                good = wait_bounded(bar_pv_done((j - 1) % C::kPBufs), (uint32_t)(((j - 1) / C::kPBufs) & 1),
+                                    abort_flag, p.wait_limit);
                 if (!__all_sync(0xffffffffu, good)) {
                     tmem_wait_st();
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float alpha = (m_cur != m_prev) ? ex2_approx(m_prev - m_cur) : 1.f;
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int q4 = 0; q4 < D / 32; ++q4) {
-                        const uint32_t ocol = tmem + lane_off + C::kColO + 32u * q4;
-                        uint32_t u[32];
-                        tmem_ld32(ocol, u);
-                        tmem_wait_ld();
+                for (int q4 = 0; q4 < D / 32; ++q4) {
+                    const uint32_t ocol = tmem + lane_off + C::kColO + 32u * q4;
+                    uint32_t u[32];
+                    tmem_ld32(ocol, u);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            reg_after_wait(u[i]);
-                            reg_after_wait(u[i + 1]);
-                            const float2 v = __fmul2_rn(
-                                make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
-                                make_float2(alpha, alpha));
-                            u[i] = __float_as_uint(v.x);
-                            u[i + 1] = __float_as_uint(v.y);
-                        }
-                        tmem_st32(ocol, u);
+                    for (int i = 0; i < 32; i += 2) {
+                        reg_after_wait(u[i]);
+                        reg_after_wait(u[i + 1]);
+                        const float2 v = __fmul2_rn(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                                    make_float2(alpha, alpha));
+                        u[i] = __float_as_uint(v.x);
+                        u[i + 1] = __float_as_uint(v.y);
                     }
+                    tmem_st32(ocol, u);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_p_full(buf));
+            if (lane == 0) mbar_arrive(bar_p_full(pb));
         }
 
         // ---------------------------------------------------------- epilogue
@@ -517,25 +554,28 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const bool have_o = n_kv > 0;
         bool good = ok;
         if (good && have_o) {
-            good = wait_bounded(bar_o_done((n_kv - 1) & 1), (uint32_t)(((n_kv - 1) >> 1) & 1), abort_flag,
-                                p.wait_limit);
+            // every MMA of the CTA is done: the drain commit completes its only phase
+            good = wait_bounded(bar_drain, 0, abort_flag, p.wait_limit);
             good = __all_sync(0xffffffffu, good);
             if (good) tc_fence_after();
         }
-        epi[par * kBlockM + r] = m_seen;
-        epi[(2 + par) * kBlockM + r] = l;
+        epi[g * kBlockM + r] = m_seen;
+        epi[(2 + g) * kBlockM + r] = l;
+        epi[(4 + g) * kBlockM + r] = lu;
         good = !named_bar_or(kBarQuadBase + qd, 64, !good);
-        // both warps' sums, brought to the final (largest) reference max
-        const float m_oth = epi[(par ^ 1) * kBlockM + r];
-        const float l_oth = epi[(2 + (par ^ 1)) * kBlockM + r];
-        const float m_fin = fmaxf(m_seen, m_oth);
-        const float l_row = (m_seen == m_fin ? l : l * ex2_approx(m_seen - m_fin)) +
-                            (m_oth == m_fin ? l_oth : l_oth * ex2_approx(m_oth - m_fin));
+        // both warps' sums, brought to the final (largest) reference max, in a
+        // fixed order so both warps get the same bits
+        const float m0w = epi[r], m1w = epi[kBlockM + r];
+        const float m_fin = fmaxf(m0w, m1w);
+        const float f0 = (m0w == m_fin) ? 1.f : ex2_approx(m0w - m_fin);
+        const float f1 = (m1w == m_fin) ? 1.f : ex2_approx(m1w - m_fin);
+        const float l_row = epi[2 * kBlockM + r] * f0 + epi[3 * kBlockM + r] * f1;    // normalises O
+        const float lu_row = epi[4 * kBlockM + r] * f0 + epi[5 * kBlockM + r] * f1;   // gives the LSE
         if (good) {
             const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
 #pragma unroll
             for (int q4 = 0; q4 < D / 64; ++q4) {
-                const int col0 = par * (D / 2) + 32 * q4;   // first O column of this chunk
+                const int col0 = g * (D / 2) + 32 * q4;   // first O column of this chunk
                 uint32_t u[32];
                 if (have_o) {
                     tmem_ld32(tmem + lane_off + C::kColO + (uint32_t)col0, u);
@@ -562,8 +602,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                                  : "memory");
                 }
             }
-            if (par == 0 && row < p.Nq) {
-                const float lse = (l_row > 0.f) ? (m_fin + lg2_approx(l_row)) * 0.69314718055994531f : -INFINITY;
+            if (g == 0 && row < p.Nq) {
+                const float lse = (lu_row > 0.f) ? (m_fin + lg2_approx(lu_row)) * 0.69314718055994531f : -INFINITY;
                 p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
             }
         }

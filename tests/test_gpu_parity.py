@@ -185,3 +185,19 @@ def test_host_entry_matches_device_entry():
 def test_device_status_is_clean_after_the_suite():
     from io_aware_exact_24_b200 import FA_OK, fa_get_device_status
     assert fa_get_device_status() == FA_OK
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rescale_path_with_growing_scores(d, causal):
+    # keys grow along the sequence, so most rows move their reference max by more
+    # than 2^8 many times: every O-rescale step (including the last tile) runs
+    B, H, N = 1, 2, 1100
+    q, k, v = _rand(B, H, N, N, d, 90 + d)
+    ramp = (1.0 + np.arange(N, dtype=np.float32) / 96.0)[None, None, :, None]
+    k = f32_to_bf16_bits(bf16_bits_to_f32(k) * ramp)
+    # one very large score in the last key tile of every row
+    k[:, :, N - 3, :] = f32_to_bf16_bits(bf16_bits_to_f32(k[:, :, N - 3, :]) * 4.0)
+    o, lse = run_fa(q, k, v, 0.5, causal, None)
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, 0.5, causal, None)
+    compare(o, lse, o_ref, lse_ref, f"growing d{d} causal={causal}")
