@@ -112,6 +112,7 @@ struct Cfg {
     // s_full[2 (per softmax warp)], s_free[2], p_full[3], pv_done[3],
     // m_ready[4 quadrants][2], drain
     static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 3 + 3 + 8 + 1;
+    static_assert(kSBufs <= 2 && kPBufs <= 3, "barrier slots");
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
     static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row]
     static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, l, lu [2][row] each
@@ -213,6 +214,7 @@ __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float 
         lu = __fadd2_rn(lu, e);
         lr = __fadd2_rn(lr, make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)));
     }
+
     tmem_st32(taddr_p + 32u * h2, w);
 }
 
