@@ -30,7 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from io_aware_exact_24_b200.inputs import WORKLOADS, WORKLOAD_ORDER, make_inputs  # noqa: E402
+from io_aware_exact_24_b200.inputs import (DECODE_WORKLOADS, WORKLOADS, WORKLOAD_ORDER,  # noqa: E402
+                                           make_inputs)
 
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -175,6 +176,60 @@ def time_device(w, x, steps, warmup, device, rank, world, clocks=None):
     return float(np.mean(per)), per, clk
 
 
+def time_splitkv(w, x, steps, warmup, device, num_splits=None):
+    """Mean per-call device time (ms) of fa_fwd_splitkv (partials + merge), L2 flushed between calls."""
+    import torch
+    from io_aware_exact_24_b200 import (fa_fwd_splitkv, fa_fwd_splitkv_workspace_size,
+                                        fa_splitkv_num_splits)
+    q, k, v, kl = upload(x, device)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    if num_splits is None:
+        num_splits = fa_splitkv_num_splits(w.B, w.H, w.Nq, w.Nk)
+    ws_bytes = fa_fwd_splitkv_workspace_size(w.B, w.H, w.Nq, w.d, num_splits)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        fa_fwd_splitkv(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
+                       num_splits, ws, ws_bytes, stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for st, en in ev:
+        flush.zero_()
+        st.record(stream)
+        launch()
+        en.record(stream)
+    torch.cuda.synchronize()
+    per = [st.elapsed_time(en) for st, en in ev]
+    del q, k, v, o, lse, flush, ws
+    return float(np.mean(per)), num_splits
+
+
+def decode_table(steps, warmup, device, hbm_gbs):
+    """Split-KV forward on the decode-shaped workloads: HBM-bound, reported in GB/s."""
+    out = {}
+    for name, w in DECODE_WORKLOADS.items():
+        x = make_inputs(w)
+        ms, ns = time_splitkv(w, x, steps, warmup, device)
+        ms1, _, _ = time_device(w, x, steps, warmup, device, 0, 1)
+        gbs = w.algorithmic_bytes / (ms / 1000.0) / 1e9
+        out[name] = {"entry": "fa_fwd_splitkv", "num_splits": ns, "ms": ms,
+                     "algorithmic_gbs": gbs, "roofline": {"bound": "hbm", "achieved": gbs,
+                                                          "peak": hbm_gbs, "unit": "GB/s",
+                                                          "frac": gbs / hbm_gbs},
+                     "single_pass_fa_fwd_ms": ms1,
+                     "config": config_of(w, "flushed between timed launches", "single GPU")}
+        del x
+    return out
+
+
 def time_e2e(w, x, steps, warmup, device):
     """The same forward through the host-buffer C entry point: H2D + kernel + D2H per step."""
     import torch
@@ -294,6 +349,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the per-workload table, e2e and CPU baseline (profiling runs)")
+    ap.add_argument("--decode", default=None, choices=sorted(DECODE_WORKLOADS),
+                    help="time only the split-KV forward on this decode workload (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -314,6 +371,19 @@ def main():
     build.build()
     load_library()
 
+    if args.decode:
+        w = DECODE_WORKLOADS[args.decode]
+        ms, ns = time_splitkv(w, make_inputs(w), args.steps, args.warmup, device)
+        peaks, peaks_src = load_peaks()
+        gbs = w.algorithmic_bytes / (ms / 1000.0) / 1e9
+        print(json.dumps({"metric": "split-KV attention fwd, algorithmic GB/s", "value": gbs,
+                          "unit": "GB/s", "ms_per_step": ms, "num_splits": ns,
+                          "roofline": {"bound": "hbm", "achieved": gbs,
+                                       "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                       "frac": gbs / float(peaks["hbm_gbs"])},
+                          "config": config_of(w, "flushed between timed launches", "single GPU")}),
+              flush=True)
+        return 0
     w = WORKLOADS[args.workload]
     x = make_inputs(w)
     clocks = ClockSampler(local)
@@ -361,6 +431,8 @@ def main():
                             "frac_of_peak": wn.flop / (ms_n / 1000.0) / 1e12 / peak,
                             "algorithmic_gbs": wn.algorithmic_bytes / (ms_n / 1000.0) / 1e9}
         line["per_workload"] = per_wl
+        line["splitkv_decode"] = decode_table(args.steps, args.warmup, device,
+                                              float(peaks["hbm_gbs"]))
         cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
         rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",

@@ -120,6 +120,61 @@ FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *o, flo
                 const int32_t *key_lens, void *workspace, size_t workspace_bytes,
                 fa_stream_t stream);
 
+/*
+ * Split-KV forward (decode-shaped problems: few query rows, long keys).
+ *
+ * Same operation, masks, layouts and outputs as fa_fwd.  The K/V tiles each
+ * 128-row query block must visit are cut into num_splits contiguous ranges;
+ * one CTA per (range, query block, head, batch) computes that range's
+ * normalised partial output O_s and log-sum-exp LSE_s into the workspace, and
+ * a second kernel merges them per row: with M = max_s LSE_s and
+ * w_s = exp(LSE_s - M), O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s
+ * (a row with no visible key in any range: O = 0, LSE = -inf).  This is the
+ * decode / FlashDecoding case "FlashAttention：把注意力从公式写成数据流"
+ * (section "端侧与专用加速器") and "[2205.14135] FlashAttention: Fast and
+ * Memory-Efficient Exact Attention with IO-Awareness" point to, merged with the
+ * same running-max rule as the online softmax ("分块与在线 softmax").  It
+ * spreads a small query batch over all SMs.
+ */
+
+/*
+ * fa_splitkv_num_splits -- a range count for this problem: 1 when the plain
+ * grid (one CTA per 128 query rows and head) already covers 4/5 of B200's 148
+ * SMs, else as many ranges as keep the grid within one wave (one CTA per SM),
+ * with at least two K/V tiles (256 keys) per range and at most 256 ranges.
+ * Returns 1 for empty or invalid sizes.  Pure host arithmetic.
+ */
+FA_API int fa_splitkv_num_splits(int B, int H, int N_q, int N_k);
+
+/*
+ * fa_fwd_splitkv_workspace_size -- bytes of device workspace fa_fwd_splitkv
+ * needs: num_splits*B*H*N_q*d fp32 partial outputs followed by
+ * num_splits*B*H*N_q fp32 partial LSEs, each 256-byte aligned.  Returns 0 for
+ * invalid sizes or num_splits outside [1, 256].
+ */
+FA_API size_t fa_fwd_splitkv_workspace_size(int B, int H, int N_q, int d, int num_splits);
+
+/*
+ * fa_fwd_splitkv -- split-KV forward on device buffers, asynchronous on `stream`.
+ *
+ *   q .. key_lens, stream   as for fa_fwd.
+ *   num_splits              1 .. 256 (more ranges than K/V tiles leaves some
+ *                           ranges empty, which is allowed).
+ *   workspace               device buffer of at least
+ *                           fa_fwd_splitkv_workspace_size(B,H,N_q,d,num_splits)
+ *                           bytes, 256-byte aligned, owned by the caller; it
+ *                           needs no initial contents.  Calls that share a
+ *                           workspace must be ordered (same stream or events).
+ *
+ * Returns what fa_fwd returns, plus FA_ERR_INVALID_ARG for num_splits out of
+ * range or a NULL / too small workspace and FA_ERR_MISALIGNED for a workspace
+ * that is not 256-byte aligned (all checked before any CUDA call).
+ */
+FA_API int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                   const int32_t *key_lens, int num_splits, void *workspace,
+                   size_t workspace_bytes, fa_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char *fa_status_string(int status);
 

@@ -60,6 +60,13 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                         i32, vp, vp, sz, vp]
             lib.fa_fwd_host.restype = i32
+            lib.fa_splitkv_num_splits.argtypes = [i32, i32, i32, i32]
+            lib.fa_splitkv_num_splits.restype = i32
+            lib.fa_fwd_splitkv_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+            lib.fa_fwd_splitkv_workspace_size.restype = sz
+            lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                           i32, vp, i32, vp, sz, vp]
+            lib.fa_fwd_splitkv.restype = i32
             lib.fa_status_string.argtypes = [i32]
             lib.fa_status_string.restype = ctypes.c_char_p
             lib.fa_get_device_status.argtypes = [vp]
@@ -116,6 +123,28 @@ def fa_fwd(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal=False, key_lens=Non
                                int(bool(causal)), _addr(key_lens), _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return st
+
+
+def fa_splitkv_num_splits(B, H, N_q, N_k) -> int:
+    return int(load_library().fa_splitkv_num_splits(int(B), int(H), int(N_q), int(N_k)))
+
+
+def fa_fwd_splitkv_workspace_size(B, H, N_q, d, num_splits) -> int:
+    return int(load_library().fa_fwd_splitkv_workspace_size(int(B), int(H), int(N_q), int(d),
+                                                             int(num_splits)))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, num_splits,
+                   workspace, workspace_bytes, stream=None, check=True) -> int:
+    """``fa_fwd_splitkv`` of include/fa.h: split-KV forward, device workspace given."""
+    st = load_library().fa_fwd_splitkv(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                       int(B), int(H), int(N_q), int(N_k), int(d),
+                                       float(scale), int(bool(causal)), _addr(key_lens),
+                                       int(num_splits), _addr(workspace), int(workspace_bytes),
+                                       _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv")
     return st
 
 

@@ -70,10 +70,16 @@ int prepare_device(int dev) {
             st.status = FA_ERR_UNSUPPORTED;
             return;
         }
-        e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  fa::Cfg<64>::kSmemBytes);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::Cfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      fa::Cfg<128>::kSmemBytes);
         if (e != cudaSuccess) {
             st.status = cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
@@ -123,9 +129,16 @@ bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d) 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Split-KV: partial results in the workspace, then the combine kernel.
+struct SplitParts {
+    int num_splits;   // 0: plain forward
+    float* o_part;
+    float* lse_part;
+};
+
 template <int D>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
-           float scale, int causal, const int32_t* key_lens, cudaStream_t stream) {
+           float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr}) {
     CUtensorMap tq, tk, tv, to;
     // With no keys the K/V maps are never read; give them a valid 1-row shape.
     const void* kp = N_k > 0 ? k : q;
@@ -147,11 +160,42 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.wait_limit = kWaitLimitCycles;
+    p.num_splits = sp.num_splits > 0 ? sp.num_splits : 1;
+    p.o_part = sp.o_part;
+    p.lse_part = sp.lse_part;
     const int rows_per_cta = fa::kBlockM;
-    dim3 grid((unsigned)((N_q + rows_per_cta - 1) / rows_per_cta), (unsigned)H, (unsigned)B);
-    fa::fa_fwd_sm100_kernel<D><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
+    const unsigned num_m = (unsigned)((N_q + rows_per_cta - 1) / rows_per_cta);
+    if (sp.num_splits <= 0) {
+        dim3 grid(num_m, (unsigned)H, (unsigned)B);
+        fa::fa_fwd_sm100_kernel<D, false><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        const cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
+    }
+    dim3 grid(num_m * (unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
+    fa::fa_fwd_sm100_kernel<D, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch (split-KV partials)", e);
+    const long long rows = (long long)B * H * N_q;
+    fa::fa_splitkv_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        sp.o_part, sp.lse_part, reinterpret_cast<__nv_bfloat16*>(o), lse, rows, sp.num_splits);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV combine)", e);
+}
+
+constexpr int kMaxSplits = 256;
+constexpr int kNumSms = 148;   // B200
+
+// Workspace of the split-KV forward: O partials, then LSE partials, 256-byte aligned.
+struct SplitLayout {
+    size_t o_part, lse_part, total;
+};
+SplitLayout split_layout(int B, int H, int N_q, int d, int num_splits) {
+    const size_t rows = (size_t)num_splits * B * H * N_q;
+    SplitLayout L{};
+    L.o_part = 0;
+    L.lse_part = (rows * d * 4 + 255) / 256 * 256;
+    L.total = L.lse_part + (rows * 4 + 255) / 256 * 256;
+    return L;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -215,6 +259,57 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s);
+}
+
+int fa_splitkv_num_splits(int B, int H, int N_q, int N_k) {
+    if (B <= 0 || H <= 0 || N_q <= 0 || N_k <= 0) return 1;
+    const long long ctas = (long long)((N_q + fa::kBlockM - 1) / fa::kBlockM) * B * H;
+    const int tiles = (N_k + fa::kBlockN - 1) / fa::kBlockN;
+    // One CTA fits per SM.  Once the plain grid covers most of the 148 SMs the
+    // K/V stream already runs at HBM speed and splitting only adds the merge;
+    // below that, split into as many ranges as still fit in one wave, with at
+    // least two K/V tiles per range.
+    if (ctas >= kNumSms * 4 / 5) return 1;
+    long long s = kNumSms / ctas;
+    const long long cap = tiles / 2 > 1 ? tiles / 2 : 1;
+    if (s > cap) s = cap;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return s < 1 ? 1 : (int)s;
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N_q, int d, int num_splits) {
+    if (B < 0 || H < 0 || N_q < 0 || (d != 64 && d != 128) || num_splits < 1 || num_splits > kMaxSplits) return 0;
+    return split_layout(B, H, N_q, d, num_splits).total;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
+                   int d, float scale, int causal, const int32_t* key_lens, int num_splits, void* workspace,
+                   size_t workspace_bytes, fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
+    if (empty) return FA_OK;
+    const SplitLayout L = split_layout(B, H, N_q, d, num_splits);
+    if (workspace == nullptr || workspace_bytes < L.total) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+    if ((unsigned long long)((N_q + fa::kBlockM - 1) / fa::kBlockM) * num_splits > 0x7fffffffull)
+        return FA_ERR_UNSUPPORTED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part)};
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }
 
 size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has_key_lens) {

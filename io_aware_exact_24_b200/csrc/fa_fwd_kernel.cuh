@@ -85,6 +85,11 @@ struct FwdParams {
     float scale_log2;           // scale * log2(e), > 0
     int causal;
     unsigned long long wait_limit;  // clock64 cycles per wait before giving up
+    // split-KV mode only: each Q tile's K/V tiles are cut into num_splits
+    // contiguous ranges, one CTA each, writing a partial result per range
+    int num_splits;
+    float* o_part;              // [num_splits, B, H, Nq, D] fp32, O of the range / its own l
+    float* lse_part;            // [num_splits, B, H, Nq] fp32, LSE of the range (-inf if empty)
 };
 
 template <int D>
@@ -236,7 +241,13 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
     return c < kl ? (int)c : kl;
 }
 
-template <int D>
+// kSplit = false: the whole forward (O and LSE).  kSplit = true: the first half
+// of the split-KV forward ("FlashAttention：把注意力从公式写成数据流", section
+// "端侧与专用加速器", and "[2205.14135] FlashAttention: Fast and
+// Memory-Efficient Exact Attention with IO-Awareness", its note on the decode
+// case): partial (O, LSE) for one contiguous range of K/V tiles, merged by
+// fa_splitkv_combine_kernel.
+template <int D, bool kSplit = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -270,9 +281,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work item: (b, h, 128-row block); heavy causal blocks launch first
-    const int num_m = (int)gridDim.x;
-    const int m_blk = p.causal ? (num_m - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    // ---- work item: (b, h, 128-row block[, K/V range]); heavy causal blocks launch first
+    const int n_split = kSplit ? p.num_splits : 1;
+    const int split = kSplit ? (int)blockIdx.x % n_split : 0;
+    const int blk = kSplit ? (int)blockIdx.x / n_split : (int)blockIdx.x;
+    const int num_m = (int)gridDim.x / n_split;
+    const int m_blk = p.causal ? (num_m - 1 - blk) : blk;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int m0 = m_blk * kBlockM;
@@ -282,9 +296,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         kl = kl < 0 ? 0 : (kl > p.Nk ? p.Nk : kl);
     }
     const int off = p.Nk - p.Nq;  // causal diagonal offset (bottom-right aligned)
-    // K/V tiles this Q tile must visit: enough for its last real row.
+    // K/V tiles this Q tile must visit: enough for its last real row; in
+    // split-KV mode this CTA takes tiles t0 .. t0+n_kv-1 of them.
     const int last_row = min(m0 + kBlockM - 1, p.Nq - 1);
-    const int n_kv = (row_key_limit(last_row, kl, off, p.causal) + kBlockN - 1) / kBlockN;
+    const int n_all = (row_key_limit(last_row, kl, off, p.causal) + kBlockN - 1) / kBlockN;
+    const int t0 = kSplit ? (int)((long long)split * n_all / n_split) : 0;
+    const int n_kv = kSplit ? (int)((long long)(split + 1) * n_all / n_split) - t0 : n_all;
 
     // ---- setup: barriers (producer lane 0), TMEM (MMA warp)
     if (warp == kProducerWarp && lane == 0) {
@@ -346,8 +363,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_full(rg, s), (uint32_t)C::kTileBytes);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64, j * kBlockN,
-                                h, b, pol_kv);
+                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64,
+                                (t0 + j) * kBlockN, h, b, pol_kv);
             }
             if (!ok) {
                 // wind down: let every copy still in flight (at most one per
@@ -456,7 +473,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_s_free(j % C::kSBufs));
-            const int kbase = j * kBlockN;
+            const int kbase = (t0 + j) * kBlockN;
             // warp-uniform: the element mask runs only on tiles that cross a row's key limit
             const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim);
             if (masked) {
@@ -588,30 +605,46 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) u[i] = 0u;
                 }
-                uint32_t pkd[16];
+                if constexpr (kSplit) {
+                    // partial O of this K/V range, fp32, straight to global memory
+                    if (row < p.Nq) {
+                        float4* dst = reinterpret_cast<float4*>(
+                            p.o_part + ((((size_t)split * p.B + b) * p.H + h) * (size_t)p.Nq + row) * D + col0);
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pkd[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-                // 4 x 16-byte chunks of row r; chunk cc of the row lives in box cc/8,
-                // swizzled position (cc%8) ^ (r%8) inside the row's 128 bytes.
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            dst[v4] = make_float4(__uint_as_float(u[4 * v4]) * inv_l, __uint_as_float(u[4 * v4 + 1]) * inv_l,
+                                                  __uint_as_float(u[4 * v4 + 2]) * inv_l,
+                                                  __uint_as_float(u[4 * v4 + 3]) * inv_l);
+                    }
+                } else {
+                    uint32_t pkd[16];
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
-                    const int cc = col0 / 8 + v4;
-                    const uint32_t addr = q_tile + (uint32_t)((cc >> 3) * kSwizzleBoxBytes + r * 128 +
-                                                              (((cc & 7) ^ (r & 7)) << 4));
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pkd[4 * v4]),
-                                 "r"(pkd[4 * v4 + 1]), "r"(pkd[4 * v4 + 2]), "r"(pkd[4 * v4 + 3])
-                                 : "memory");
+                    for (int i = 0; i < 16; ++i)
+                        pkd[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+                    // 4 x 16-byte chunks of row r; chunk cc of the row lives in box cc/8,
+                    // swizzled position (cc%8) ^ (r%8) inside the row's 128 bytes.
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const int cc = col0 / 8 + v4;
+                        const uint32_t addr = q_tile + (uint32_t)((cc >> 3) * kSwizzleBoxBytes + r * 128 +
+                                                                  (((cc & 7) ^ (r & 7)) << 4));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pkd[4 * v4]),
+                                     "r"(pkd[4 * v4 + 1]), "r"(pkd[4 * v4 + 2]), "r"(pkd[4 * v4 + 3])
+                                     : "memory");
+                    }
                 }
             }
             if (g == 0 && row < p.Nq) {
                 const float lse = (lu_row > 0.f) ? (m_fin + lg2_approx(lu_row)) * 0.69314718055994531f : -INFINITY;
-                p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
+                if constexpr (kSplit)
+                    p.lse_part[(((size_t)split * p.B + b) * p.H + h) * (size_t)p.Nq + row] = lse;
+                else
+                    p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
             }
         }
         fence_proxy_async_smem();
         const bool any_bad = named_bar_or(kBarSoftmaxAll, kSoftmaxWarps * 32, !good);
-        if (!any_bad && threadIdx.x == 0) {
+        if (!kSplit && !any_bad && threadIdx.x == 0) {
             for (int bx = 0; bx < C::kBoxes; ++bx)
                 tma_store_4d(&tm_o, q_tile + bx * kSwizzleBoxBytes, bx * 64, m0, h, b);
             bulk_commit_group();
@@ -625,6 +658,71 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// Second half of the split-KV forward: merge the partial results of the
+// K/V ranges of every query row.  With M = max_s LSE_s and w_s = e^(LSE_s - M):
+//   O = sum_s w_s O_s / sum_s w_s,   LSE = M + ln sum_s w_s
+// (each O_s is normalised by its own range's sum, so w_s carries that sum).
+// A row whose ranges are all empty (M = -inf) gets O = 0, LSE = -inf; an empty
+// range has LSE_s = -inf, so w_s = 0 and its O_s (zeros) adds nothing.
+// One warp per row; lane s holds the weights of ranges s, s+32, ...; each lane
+// owns D/32 consecutive output columns.
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_splitkv_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                              __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long rows, int n_split) {
+    constexpr int kCols = D / 32;
+    constexpr int kMaxPerLane = 8;   // n_split <= 256
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float ls[kMaxPerLane];
+    float m = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < kMaxPerLane; ++t) {
+        const int sp = lane + 32 * t;
+        ls[t] = (sp < n_split) ? lse_part[(size_t)sp * rows + row] : -INFINITY;
+        m = fmaxf(m, ls[t]);
+    }
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sh));
+    float wl[kMaxPerLane];
+    float wsum = 0.f;
+#pragma unroll
+    for (int t = 0; t < kMaxPerLane; ++t) {
+        wl[t] = (m == -INFINITY || ls[t] == -INFINITY) ? 0.f : expf(ls[t] - m);
+        wsum += wl[t];
+    }
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, sh);
+    float acc[kCols];
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+    const float* src = o_part + (size_t)row * D + lane * kCols;
+    const size_t split_stride = (size_t)rows * D;
+#pragma unroll
+    for (int t = 0; t < kMaxPerLane; ++t) {
+        if (32 * t >= n_split) break;
+#pragma unroll 4
+        for (int k2 = 0; k2 < 32; ++k2) {
+            const int sp = 32 * t + k2;
+            if (sp >= n_split) break;
+            const float w = __shfl_sync(0xffffffffu, wl[t], k2);
+            const float* p2 = src + (size_t)sp * split_stride;
+#pragma unroll
+            for (int i = 0; i < kCols; i += 2) {
+                const float2 v = *reinterpret_cast<const float2*>(p2 + i);
+                acc[i] = fmaf(w, v.x, acc[i]);
+                acc[i + 1] = fmaf(w, v.y, acc[i + 1]);
+            }
+        }
+    }
+    const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(o + row * D + lane * kCols);
+#pragma unroll
+    for (int i = 0; i < kCols; i += 2) dst[i / 2] = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+    if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
 }
 
 }  // namespace fa

@@ -81,6 +81,18 @@ WORKLOADS = {
 WORKLOAD_ORDER = ["tiny", "gpt2_causal_1k", "bert_padded_512", "long_16k_d64",
                   "causal_8000_d128"]
 
+# Decode-shaped problems for the split-KV forward: one query row per (b, h)
+# against a long key sequence (the inference case FlashAttention's long-sequence
+# discussion leads to).  K and V (1.07 GB) are far larger than L2, so these
+# measure the HBM stream.
+DECODE_WORKLOADS = {
+    "decode_16k_d128": Workload("decode_16k_d128", 4, 32, 1, 16384, 128, False,
+                                float(np.float32(1 / math.sqrt(128))), 1.0, None, 6),
+    # few heads: 8 query blocks cannot fill the GPU without splitting the keys
+    "decode_64k_h8_d128": Workload("decode_64k_h8_d128", 1, 8, 1, 65536, 128, False,
+                                   float(np.float32(1 / math.sqrt(128))), 1.0, None, 7),
+}
+
 
 def _rng(seed: int, tensor_id: int) -> np.random.Generator:
     return np.random.Generator(np.random.Philox(key=int(seed) * 16 + int(tensor_id)))

@@ -123,3 +123,62 @@ def test_without_a_gpu_valid_calls_report_no_device(lib):
         pytest.skip("a GPU is present")
     assert call() == binding.FA_ERR_NO_DEVICE
     assert binding.fa_get_device_status(0) == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- split-KV entry points
+
+def test_splitkv_workspace_size_formula(lib):
+    for B, H, Nq, d, S in ((1, 1, 1, 64, 1), (2, 3, 5, 128, 7), (4, 32, 1, 128, 16)):
+        rows = S * B * H * Nq
+        need = binding.fa_fwd_splitkv_workspace_size(B, H, Nq, d, S)
+        o_bytes = -(-rows * d * 4 // 256) * 256
+        assert need == o_bytes + -(-rows * 4 // 256) * 256
+    assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 96, 2) == 0
+    assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 0) == 0
+    assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 257) == 0
+    assert binding.fa_fwd_splitkv_workspace_size(-1, 1, 1, 64, 2) == 0
+
+
+def test_splitkv_num_splits_heuristic(lib):
+    # few query blocks and many key tiles: spread over the SMs, >= 2 tiles per range
+    assert binding.fa_splitkv_num_splits(1, 1, 1, 1 << 20) == 148
+    assert binding.fa_splitkv_num_splits(1, 8, 1, 16384) == 18      # 144 CTAs: one wave
+    assert binding.fa_splitkv_num_splits(1, 8, 1, 1024) == 4        # 8 tiles -> ranges of >= 2
+    assert binding.fa_splitkv_num_splits(1, 1, 1, 300) == 1         # 3 tiles -> ranges of >= 2
+    assert binding.fa_splitkv_num_splits(1, 70, 1, 8192) == 2
+    assert binding.fa_splitkv_num_splits(1, 100, 1, 8192) == 1
+    assert binding.fa_splitkv_num_splits(4, 32, 1, 16384) == 1      # 128 CTAs fill the GPU
+    assert binding.fa_splitkv_num_splits(8, 32, 128, 8192) == 1
+    assert binding.fa_splitkv_num_splits(0, 1, 1, 100) == 1
+
+
+def splitkv_call(num_splits=4, ws=P, ws_bytes=1 << 30, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0,
+             key_lens=None)
+    a.update(kw)
+    return binding.fa_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                                  a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                                  a["key_lens"], num_splits, ws, ws_bytes, stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_splits=0), binding.FA_ERR_INVALID_ARG),
+    (dict(num_splits=257), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=None), binding.FA_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=P + 128), binding.FA_ERR_MISALIGNED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(q=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(num_splits=0, B=0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0, ws=None), binding.FA_OK),
+])
+def test_splitkv_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert splitkv_call(**kw) == code
+
+
+def test_splitkv_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert splitkv_call() == binding.FA_ERR_NO_DEVICE
