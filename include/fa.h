@@ -175,6 +175,30 @@ FA_API int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, 
                    const int32_t *key_lens, int num_splits, void *workspace,
                    size_t workspace_bytes, fa_stream_t stream);
 
+/*
+ * fa_fwd_splitkv_noalloc -- fa_fwd_splitkv for callers that cannot allocate
+ * device memory: the same kernels, with the workspace taken from a scratch
+ * array the library holds in a file-scope device variable of 16 MiB
+ * (16777216 bytes) per device, sized when the library's module loads.  The
+ * paper has no counterpart: this is a library convenience, not part of the
+ * method.
+ *
+ *   q .. key_lens, num_splits, stream   as for fa_fwd_splitkv.
+ *
+ * Returns what fa_fwd_splitkv returns, except that a problem whose workspace
+ * (fa_fwd_splitkv_workspace_size) exceeds 16 MiB is rejected with
+ * FA_ERR_UNSUPPORTED before any CUDA call.  Nothing in the scratch needs to
+ * start at zero.  All calls on one device share the one scratch array: calls
+ * must not overlap in time (issue them on one stream, or order them with
+ * events); two calls running concurrently on different streams corrupt each
+ * other's partial results.  The first call on each device looks up the
+ * scratch address and sets kernel attributes (host-side setup, no stream
+ * work): make that first call outside any stream capture.
+ */
+FA_API int fa_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                           int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                           const int32_t *key_lens, int num_splits, fa_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char *fa_status_string(int status);
 

@@ -67,6 +67,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                            i32, vp, i32, vp, sz, vp]
             lib.fa_fwd_splitkv.restype = i32
+            lib.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                   f32, i32, vp, i32, vp]
+            lib.fa_fwd_splitkv_noalloc.restype = i32
             lib.fa_status_string.argtypes = [i32]
             lib.fa_status_string.restype = ctypes.c_char_p
             lib.fa_get_device_status.argtypes = [vp]
@@ -145,6 +148,18 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, 
                                        _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_splitkv")
+    return st
+
+
+def fa_fwd_splitkv_noalloc(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens,
+                           num_splits, stream=None, check=True) -> int:
+    """``fa_fwd_splitkv_noalloc`` of include/fa.h: split-KV forward on the library's own scratch."""
+    st = load_library().fa_fwd_splitkv_noalloc(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                               int(B), int(H), int(N_q), int(N_k), int(d),
+                                               float(scale), int(bool(causal)), _addr(key_lens),
+                                               int(num_splits), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv_noalloc")
     return st
 
 

@@ -312,6 +312,78 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of fa_fwd_splitkv_noalloc: one file-scope device array per process
+// and device, sized once at module load (no allocation call at any time).
+constexpr size_t kNoAllocScratchBytes = 16u << 20;
+static __device__ __align__(256) unsigned char g_splitkv_scratch[kNoAllocScratchBytes];
+
+struct ScratchState {
+    std::once_flag once;
+    int status = FA_OK;
+    void* ptr = nullptr;
+};
+ScratchState g_scratch[kMaxDevices];
+
+// Device address of the scratch array on `dev`, looked up once per device.
+int scratch_address(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    ScratchState& st = g_scratch[dev];
+    std::call_once(st.once, [&] {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_splitkv_scratch);
+        if (e != cudaSuccess) {
+            st.status = cuda_fail("cudaGetSymbolAddress(split-KV scratch)", e);
+            return;
+        }
+        st.ptr = p;
+        st.status = FA_OK;
+    });
+    *out = st.ptr;
+    return st.status;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q,
+                           int N_k, int d, float scale, int causal, const int32_t* key_lens, int num_splits,
+                           fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
+    if (empty) return FA_OK;
+    const SplitLayout L = split_layout(B, H, N_q, d, num_splits);
+    if (L.total > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+    if ((unsigned long long)((N_q + fa::kBlockM - 1) / fa::kBlockM) * num_splits > 0x7fffffffull)
+        return FA_ERR_UNSUPPORTED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    void* scratch = nullptr;
+    st = scratch_address(dev, &scratch);
+    if (st != FA_OK) return st;
+    // Every partial the merge reads is written first, so nothing in the
+    // scratch has to start at zero.
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(scratch);
+    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part)};
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
+}
+
 size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has_key_lens) {
     if (B < 0 || H < 0 || N_q < 0 || N_k < 0 || (d != 64 && d != 128)) return 0;
     return host_layout(B, H, N_q, N_k, d, has_key_lens).total;
