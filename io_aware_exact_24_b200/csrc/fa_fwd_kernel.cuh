@@ -34,6 +34,9 @@
 //    between the two warps (shared memory + an mbarrier); each keeps its own
 //    partial row sums.  Exponentials are taken in the exp2 domain, some on
 //    MUFU and some with a polynomial on the FMA pipe;
+//  * V is extended by a column block of ones, so the PV product also
+//    accumulates the row sums of the bf16 P it uses (next to O, in TMEM, and
+//    rescaled with it); the softmax keeps only the unrounded sum for the LSE;
 //  * the reference max moves only when the row max grows by more than 2^8;
 //    O is then rescaled in TMEM (exact: m, l and O always share one max);
 //  * epilogue: O / l -> bf16 -> shared memory (128B-swizzled) -> TMA store
@@ -97,21 +100,26 @@ struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kBoxes = D / 64;                        // 64-column boxes per row
     static constexpr int kTileBytes = kBlockM * D * 2;           // one Q / K / V tile
-    static constexpr int kStagesK = (D == 64) ? 6 : 3;           // K ring slots
-    static constexpr int kStagesV = (D == 64) ? 6 : 2;           // V ring slots
+    static constexpr int kStagesK = (D == 64) ? 4 : 2;           // K ring slots
+    static constexpr int kStagesV = (D == 64) ? 4 : 2;           // V ring slots
+    // A V slot holds the tile (kBoxes 64-column boxes) followed by one box of
+    // bf16 ones: the PV product runs with N = D + 16 and its last 16 output
+    // columns accumulate the row sums of the bf16 P it multiplies.
+    static constexpr int kVSlotBytes = kTileBytes + kSwizzleBoxBytes;
+    static constexpr int kNPV = D + 16;
     static constexpr int kStages = kStagesK + kStagesV;
     // Of every 8 pairs of probabilities, this many are computed on the FMA pipe
     // (exp2_fma2) and the rest on MUFU, so neither unit is the lone bottleneck.
 #ifdef FA_EMU_PAIRS_D64
     static constexpr int kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
 #else
-    static constexpr int kEmuPairs = 1;
+    static constexpr int kEmuPairs = (D == 64) ? 2 : 0;   // measured best on B200
 #endif
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kTileBytes;
     static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
-    static constexpr int kBarOff = kVOff + kStagesV * kTileBytes;
-    static constexpr int kSBufs = (D == 64) ? 2 : 1;             // TMEM score buffers
+    static constexpr int kBarOff = kVOff + kStagesV * kVSlotBytes;
+    static constexpr int kSBufs = 1;                             // TMEM score buffers
     static constexpr int kPBufs = 3;                             // TMEM probability buffers
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
     // s_full[2 (per softmax warp)], s_free[2], p_full[3], pv_done[3],
@@ -120,24 +128,26 @@ struct Cfg {
     static_assert(kSBufs <= 2 && kPBufs <= 3, "barrier slots");
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
     static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row]
-    static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, l, lu [2][row] each
-    static constexpr int kSmemBytes = kEpiOff + 3 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
+    static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, lu [2][row] each
+    static constexpr int kSmemBytes = kEpiOff + 2 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
-    // TMEM columns: S buffers from 0 (128 each), then the P buffers (bf16
-    // pairs, 64 each), O in the last D columns.
-    //   D = 128: S 0..127, P 128..319, O 384..511
-    //   D = 64:  S 0..255, P 256..447, O 448..511
+    // TMEM columns: the S buffer at 0..127, the P buffers (bf16 pairs, 64
+    // each) at 128..319, O at 320..320+D-1 and its row-sum columns right
+    // after (320+D .. 320+D+15); the O rescale also touches the 16 unused
+    // columns after those (at most column 479).
     __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
     __host__ __device__ static constexpr uint32_t col_p(int b) { return 128u * kSBufs + 64u * b; }
-    static constexpr uint32_t kColO = 512u - D;
-    static_assert(128 * kSBufs + 64 * kPBufs <= 512 - D, "TMEM columns");
+    static constexpr uint32_t kColO = 128u * kSBufs + 64u * kPBufs;
+    static constexpr uint32_t kColL = kColO + D;                 // row sum of the bf16 P
+    static_assert(kColO + D + 32 <= 512, "TMEM columns");
     // Instruction descriptors (kind::f16): D=f32, A=B=bf16, M=128.
-    //   QK^T: A=Q K-major, B=K K-major, N=128.  PV: A=P (TMEM, K-major), B=V MN-major, N=D.
+    //   QK^T: A=Q K-major, B=K K-major, N=128.
+    //   PV: A=P (TMEM, K-major), B=[V | ones] MN-major, N=D+16.
     static constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
                                          (0u << 16) | ((uint32_t)(kBlockN >> 3) << 17) |
                                          ((uint32_t)(kBlockM >> 4) << 24);
     static constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
-                                         (1u << 16) | ((uint32_t)(D >> 3) << 17) |
+                                         (1u << 16) | ((uint32_t)(kNPV >> 3) << 17) |
                                          ((uint32_t)(kBlockM >> 4) << 24);
 };
 
@@ -193,14 +203,14 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 // p = 2^(s*c - mu) for keys 64*h2 .. 64*h2+63 of the thread's row, packed to
-// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2.  Two row sums: lr
-// adds the bf16-rounded p (the weights the PV product uses, so O is normalised
-// consistently), lu the unrounded p (for the log-sum-exp).  kEmu of every 8
-// pairs go through exp2_fma2, the rest through MUFU ex2 (which maps -inf to 0,
-// so masked tiles use kEmu = 0).
+// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2.  lu sums the
+// unrounded p (for the log-sum-exp; the sum of the bf16-rounded p, which
+// normalises O, comes out of the PV product).  kEmu of every 8 pairs go
+// through exp2_fma2, the rest through MUFU ex2 (which maps -inf to 0, so masked
+// tiles use kEmu = 0).
 template <int kEmu, int h2>
 __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float c, float mu, uint32_t taddr_p,
-                                               float2& lr, float2& lu) {
+                                               float2& lu) {
     const float2 c2 = make_float2(c, c);
     const float2 nmu = make_float2(-mu, -mu);
     uint32_t w[32];
@@ -217,7 +227,6 @@ __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float 
         }
         w[i] = pack_bf16x2(e.x, e.y);
         lu = __fadd2_rn(lu, e);
-        lr = __fadd2_rn(lr, make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)));
     }
 
     tmem_st32(taddr_p + 32u * h2, w);
@@ -275,7 +284,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     float* const epi = reinterpret_cast<float*>(base_ptr + C::kEpiOff);       // m, l, lu [group][row] each
     const uint32_t q_tile = base + C::kQOff;
     auto ring_slot = [&](int r, int s) {
-        return base + (r == 0 ? C::kKOff : C::kVOff) + (uint32_t)(s * C::kTileBytes);
+        return r == 0 ? base + C::kKOff + (uint32_t)(s * C::kTileBytes)
+                      : base + C::kVOff + (uint32_t)(s * C::kVSlotBytes);
     };
 
     const int warp = threadIdx.x >> 5;
@@ -333,6 +343,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tmem_relinquish();
         tc_fence_before();
     }
+    // the ones box of every V slot (TMA writes only the boxes before it)
+    for (int i = threadIdx.x; i < C::kStagesV * (kSwizzleBoxBytes / 16); i += kNumThreads) {
+        const int sl = i / (kSwizzleBoxBytes / 16);
+        const uint32_t a = ring_slot(1, sl) + (uint32_t)C::kTileBytes + (uint32_t)(i % (kSwizzleBoxBytes / 16)) * 16u;
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0x3F803F80u) : "memory");
+    }
+    fence_proxy_async_smem();   // visible to the tensor core's reads
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
@@ -443,7 +460,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int lim = row_key_limit(row, kl, off, p.causal);
         const float c = p.scale_log2;
         float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
-        float l = 0.f;             // this warp's rounded probabilities, relative to m_seen
         float lu = 0.f;            // the same sum before rounding (for the LSE)
         bool ok = true;
 
@@ -503,7 +519,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             }
             if (m_cur != m_seen) {
                 const float f = ex2_approx(m_seen - m_cur);  // 0 while m_seen is -inf
-                l *= f;
                 lu *= f;
                 m_seen = m_cur;
             }
@@ -518,16 +533,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     break;
                 }
             }
-            float2 lr2 = make_float2(0.f, 0.f), lu2 = make_float2(0.f, 0.f);
+            float2 lu2 = make_float2(0.f, 0.f);
             const uint32_t taddr_p = tmem + lane_off + C::col_p(pb);
             if (masked) {
-                exp_store_half<0, 0>(s, c, mu, taddr_p, lr2, lu2);
-                exp_store_half<0, 1>(s, c, mu, taddr_p, lr2, lu2);
+                exp_store_half<0, 0>(s, c, mu, taddr_p, lu2);
+                exp_store_half<0, 1>(s, c, mu, taddr_p, lu2);
             } else {
-                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, lr2, lu2);
-                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, lr2, lu2);
+                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, lu2);
+                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, lu2);
             }
-            l += lr2.x + lr2.y;
             lu += lu2.x + lu2.y;
             // O holds tiles < j relative to m_prev.  Only when some row of this
             // warp moved its reference max does O have to be rescaled, and only
@@ -544,7 +558,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll
-                for (int q4 = 0; q4 < D / 32; ++q4) {
+                for (int q4 = 0; q4 < D / 32 + 1; ++q4) {   // O and its row-sum columns
                     const uint32_t ocol = tmem + lane_off + C::kColO + 32u * q4;
                     uint32_t u[32];
                     tmem_ld32(ocol, u);
@@ -579,8 +593,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             if (good) tc_fence_after();
         }
         epi[g * kBlockM + r] = m_seen;
-        epi[(2 + g) * kBlockM + r] = l;
-        epi[(4 + g) * kBlockM + r] = lu;
+        epi[(2 + g) * kBlockM + r] = lu;
         good = !named_bar_or(kBarQuadBase + qd, 64, !good);
         // both warps' sums, brought to the final (largest) reference max, in a
         // fixed order so both warps get the same bits
@@ -588,9 +601,18 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const float m_fin = fmaxf(m0w, m1w);
         const float f0 = (m0w == m_fin) ? 1.f : ex2_approx(m0w - m_fin);
         const float f1 = (m1w == m_fin) ? 1.f : ex2_approx(m1w - m_fin);
-        const float l_row = epi[2 * kBlockM + r] * f0 + epi[3 * kBlockM + r] * f1;    // normalises O
-        const float lu_row = epi[4 * kBlockM + r] * f0 + epi[5 * kBlockM + r] * f1;   // gives the LSE
+        const float lu_row = epi[2 * kBlockM + r] * f0 + epi[3 * kBlockM + r] * f1;   // gives the LSE
         if (good) {
+            // O and the sum of the bf16 P it was built from share every rescale,
+            // so O / l needs no reference max
+            float l_row = 0.f;
+            if (have_o) {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_off + C::kColL, u);
+                tmem_wait_ld();
+                reg_after_wait(u[0]);
+                l_row = __uint_as_float(u[0]);
+            }
             const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
 #pragma unroll
             for (int q4 = 0; q4 < D / 64; ++q4) {
