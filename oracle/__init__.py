@@ -63,6 +63,9 @@ def _load():
             lib.attn_ref_fp64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                           f32, i32, vp, vp, vp]
             lib.attn_ref_fp64.restype = i32
+            lib.attn_ref_fp64_window.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                                 f32, i32, i64, vp, vp, vp]
+            lib.attn_ref_fp64_window.restype = i32
             lib.attn_ref_fp64_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
                                                i64, f32, i32, vp, i64, vp, vp]
             lib.attn_ref_fp64_rows.restype = i32
@@ -112,6 +115,20 @@ def attn_ref(q, k, v, scale, causal=False, key_lens=None, return_p=False):
     if rc != 0:
         raise RuntimeError(f"attn_ref_fp64 failed ({rc})")
     return (o, lse, p) if return_p else (o, lse)
+
+
+def attn_ref_window(q, k, v, scale, window_left, causal=False, key_lens=None):
+    """Plain definition with a sliding window of window_left keys before each
+    row's diagonal position.  Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq])."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    o = np.empty((B, H, Nq, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    rc = _load().attn_ref_fp64_window(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
+                                      Nq, Nk, d, float(np.float32(scale)), int(bool(causal)),
+                                      int(window_left), _ptr(o), _ptr(lse), None)
+    if rc != 0:
+        raise RuntimeError(f"attn_ref_fp64_window failed ({rc})")
+    return o, lse
 
 
 def attn_ref_rows(q, k, v, scale, row_ids, causal=False, key_lens=None):

@@ -21,6 +21,12 @@
  *   - both masks combine with AND; the valid keys of row i are therefore the
  *     prefix [0, lim_i);
  *   - a row with no valid key has O = 0 and LSE = -inf.
+ *   - sliding window (attn_ref_fp64_window only): with window_left = W >= 0
+ *     key j is also masked when j < i + (N_k - N_q) - W, so row i sees the
+ *     keys [lo_i, lim_i), lo_i = max(0, i + N_k - N_q - W): at most the W
+ *     keys before its diagonal position plus that position.  This is the
+ *     local-attention mask of the "mask variants" the second page's section
+ *     "精度、掩码和边界情况" groups with causal and padding masks.
  *
  * Nothing here is shared with the CUDA path.  Only tests/, the package's
  * graft entry smoke check and bench.py's CPU baseline may call it.
@@ -67,18 +73,25 @@ static int64_t row_limit(int64_t i, int64_t b, const int32_t *key_lens,
     return lim;
 }
 
+/* First valid key of row i under a sliding window of W keys (W < 0: none). */
+static int64_t row_start(int64_t i, int64_t Nq, int64_t Nk, int64_t W) {
+    if (W < 0) return 0;
+    int64_t lo = i + (Nk - Nq) - W;
+    return lo < 0 ? 0 : lo;
+}
+
 /*
- * One query row, straight from the definition.  s_row and p_row are caller
- * scratch of length Nk; on return they hold S_i (masked entries -inf) and
- * P_i (masked entries 0).
+ * One query row, straight from the definition.  The valid keys are
+ * [lo, lim).  s_row and p_row are caller scratch of length Nk; on return they
+ * hold S_i (masked entries -inf) and P_i (masked entries 0).
  */
 static void one_row(const uint16_t *q_row, const uint16_t *k_head,
                     const uint16_t *v_head, int64_t Nk, int64_t d,
-                    double scale, int64_t lim, double *s_row, double *p_row,
+                    double scale, int64_t lo, int64_t lim, double *s_row, double *p_row,
                     double *o_row, double *lse_out) {
     /* S_ij = scale * sum_c q_ic k_jc for valid j, -inf for masked j. */
     for (int64_t j = 0; j < Nk; ++j) {
-        if (j < lim) {
+        if (j >= lo && j < lim) {
             double dot = 0.0;
             for (int64_t c = 0; c < d; ++c)
                 dot += bf16_bits_to_f64(q_row[c]) * bf16_bits_to_f64(k_head[j * d + c]);
@@ -87,7 +100,7 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
             s_row[j] = -INFINITY;
         }
     }
-    if (lim == 0) {
+    if (lim <= lo) {
         for (int64_t j = 0; j < Nk; ++j) p_row[j] = 0.0;
         for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
         *lse_out = -INFINITY;
@@ -95,17 +108,17 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
     }
     /* softmax over the valid entries: subtract the row max, exp, normalise. */
     double m = -INFINITY;
-    for (int64_t j = 0; j < lim; ++j)
+    for (int64_t j = lo; j < lim; ++j)
         if (s_row[j] > m) m = s_row[j];
     double l = 0.0;
     for (int64_t j = 0; j < Nk; ++j) {
-        p_row[j] = (j < lim) ? exp(s_row[j] - m) : 0.0;
+        p_row[j] = (j >= lo && j < lim) ? exp(s_row[j] - m) : 0.0;
         l += p_row[j];
     }
     for (int64_t j = 0; j < Nk; ++j) p_row[j] /= l;
     /* O_i = sum_j P_ij V_j */
     for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
-    for (int64_t j = 0; j < lim; ++j)
+    for (int64_t j = lo; j < lim; ++j)
         for (int64_t c = 0; c < d; ++c)
             o_row[c] += p_row[j] * bf16_bits_to_f64(v_head[j * d + c]);
     *lse_out = m + log(l);
@@ -118,10 +131,15 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
  * scale is the fp32 value the GPU receives, widened to fp64.
  * Returns 0, or -1 on bad sizes / allocation failure.
  */
-int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                  const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                  int64_t Nk, int64_t d, float scale, int causal, double *o,
-                  double *lse, double *p_out) {
+/*
+ * Sliding-window forward (window_left = W >= 0 keys before the diagonal
+ * position, see the header comment; W < 0 means no window and gives exactly
+ * attn_ref_fp64).  Arguments otherwise as attn_ref_fp64.
+ */
+int attn_ref_fp64_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                         int64_t Nk, int64_t d, float scale, int causal,
+                         int64_t window_left, double *o, double *lse, double *p_out) {
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0) return -1;
     const double sc = (double)scale;
     const int64_t rows = B * H * Nq;
@@ -140,8 +158,9 @@ int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const int64_t bh = r / Nq;
                 const int64_t b = bh / H;
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
+                const int64_t lo = row_start(i, Nq, Nk, window_left);
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        lim, s_row, p_row, o + r * d, lse + r);
+                        lo, lim, s_row, p_row, o + r * d, lse + r);
                 if (p_out) memcpy(p_out + r * Nk, p_row, sizeof(double) * (size_t)Nk);
             }
         }
@@ -149,6 +168,14 @@ int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         free(p_row);
     }
     return failed ? -1 : 0;
+}
+
+int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                  int64_t Nk, int64_t d, float scale, int causal, double *o,
+                  double *lse, double *p_out) {
+    return attn_ref_fp64_window(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, -1,
+                                o, lse, p_out);
 }
 
 /*
@@ -183,7 +210,7 @@ int attn_ref_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const int64_t b = bh / H;
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        lim, s_row, p_row, o_rows + t * d, lse_rows + t);
+                        0, lim, s_row, p_row, o_rows + t * d, lse_rows + t);
             }
         }
         free(s_row);

@@ -249,3 +249,66 @@ def test_rows_entry_matches_full_evaluation():
     orow, lrow = oracle.attn_ref_rows(q, k, v, 0.125, rows, True, kl)
     assert np.array_equal(orow, o.reshape(-1, d)[rows])
     assert np.array_equal(lrow, lse.reshape(-1)[rows])
+
+
+# ---------------------------------------------------------------- sliding window
+
+WINDOW_CASES = [
+    # B, H, Nq, Nk, d, causal, key_lens, W
+    (1, 2, 9, 9, 8, True, None, 3),
+    (2, 1, 7, 12, 16, True, [12, 5], 2),
+    (1, 1, 12, 5, 8, True, None, 1),      # N_q > N_k: leading rows see nothing
+    (2, 2, 6, 10, 8, False, [3, 10], 4),  # non-causal: only the lower bound applies
+    (1, 1, 16, 16, 4, True, None, 0),
+]
+
+
+def _window_rows(Nq, Nk, causal, kl, W):
+    lo = [max(0, i + Nk - Nq - W) for i in range(Nq)]
+    hi = [min(kl, i + Nk - Nq + 1) if causal else kl for i in range(Nq)]
+    return lo, [max(h, 0) for h in hi]
+
+
+@pytest.mark.parametrize("case", WINDOW_CASES)
+def test_window_equals_plain_attention_on_the_key_slice(case):
+    # a window only removes keys: each row equals the plain (unmasked) definition
+    # evaluated on its own slice [lo, hi) of K and V
+    B, H, Nq, Nk, d, causal, kl, W = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 31)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o, lse = oracle.attn_ref_window(q, k, v, 0.3, W, causal, kl_arr)
+    for b in range(B):
+        lo, hi = _window_rows(Nq, Nk, causal, Nk if kl is None else kl[b], W)
+        for h in range(H):
+            for i in range(Nq):
+                if hi[i] <= lo[i]:
+                    assert np.all(o[b, h, i] == 0) and np.isneginf(lse[b, h, i])
+                    continue
+                sl = slice(lo[i], hi[i])
+                o1, l1 = oracle.attn_ref(q[b:b + 1, h:h + 1, i:i + 1], k[b:b + 1, h:h + 1, sl],
+                                         v[b:b + 1, h:h + 1, sl], 0.3, False, None)
+                np.testing.assert_allclose(o[b, h, i], o1[0, 0, 0], rtol=0, atol=1e-13)
+                assert abs(lse[b, h, i] - l1[0, 0, 0]) <= 1e-13
+
+
+def test_window_zero_sees_only_the_diagonal_key():
+    # W = 0 with causal and N_q = N_k: row i sees key i alone, so O_i = V_i and
+    # LSE_i = scale * q_i . k_i exactly (closed form)
+    q, k, v = _rand(2, 2, 11, 11, 8, 32)
+    o, lse = oracle.attn_ref_window(q, k, v, 0.25, 0, True, None)
+    qf, kf, vf = (bf16_bits_to_f32(x).astype(np.float64) for x in (q, k, v))
+    assert np.array_equal(o, vf)
+    s_diag = np.einsum("bhid,bhid->bhi", qf, kf) * float(np.float32(0.25))
+    np.testing.assert_allclose(lse, s_diag, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_wide_window_is_no_window(causal):
+    q, k, v = _rand(2, 3, 13, 17, 8, 33)
+    kl = np.array([17, 9], np.int32)
+    o0, l0 = oracle.attn_ref(q, k, v, 0.2, causal, kl)
+    for W in (17, 40):
+        o1, l1 = oracle.attn_ref_window(q, k, v, 0.2, W, causal, kl)
+        assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+    o2, l2 = oracle.attn_ref_window(q, k, v, 0.2, -1, causal, kl)
+    assert np.array_equal(o0, o2) and np.array_equal(l0, l2)
