@@ -30,8 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from io_aware_exact_24_b200.inputs import (DECODE_WORKLOADS, WORKLOADS, WORKLOAD_ORDER,  # noqa: E402
-                                           make_inputs)
+from io_aware_exact_24_b200.inputs import (DECODE_WORKLOADS, WINDOW_WORKLOADS,  # noqa: E402
+                                           WORKLOADS, WORKLOAD_ORDER, make_inputs)
 
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -174,6 +174,51 @@ def time_device(w, x, steps, warmup, device, rank, world, clocks=None):
     per = [s.elapsed_time(e) for s, e in ev]
     del q, k, v, o, lse, flush
     return float(np.mean(per)), per, clk
+
+
+def time_window(w, x, steps, warmup, device):
+    """Mean per-call device time (ms) of fa_fwd_window, L2 flushed between calls."""
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd_window
+    q, k, v, kl = upload(x, device)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        fa_fwd_window(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
+                      w.window_left, stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for st, en in ev:
+        flush.zero_()
+        st.record(stream)
+        fa_fwd_window(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
+                      w.window_left, stream)
+        en.record(stream)
+    torch.cuda.synchronize()
+    per = [st.elapsed_time(en) for st, en in ev]
+    del q, k, v, o, lse, flush
+    return float(np.mean(per))
+
+
+def window_table(steps, warmup, device, peak_tflops):
+    """Sliding-window forward: TFLOP/s on the visible (query, key) pairs only."""
+    out = {}
+    for name, w in WINDOW_WORKLOADS.items():
+        x = make_inputs(w)
+        ms = time_window(w, x, steps, warmup, device)
+        tf = w.flop / (ms / 1000.0) / 1e12
+        out[name] = {"entry": "fa_fwd_window", "window_left": w.window_left, "ms": ms,
+                     "tflops": tf, "roofline": {"bound": "tensor", "achieved": tf,
+                                                "peak": peak_tflops, "unit": "TFLOP/s",
+                                                "frac": tf / peak_tflops},
+                     "flop": "4*B*H*d*(visible query-key pairs)",
+                     "config": config_of(w, "flushed between timed launches", "single GPU")}
+        del x
+    return out
 
 
 def time_splitkv(w, x, steps, warmup, device, num_splits=None):
@@ -433,6 +478,7 @@ def main():
         line["per_workload"] = per_wl
         line["splitkv_decode"] = decode_table(args.steps, args.warmup, device,
                                               float(peaks["hbm_gbs"]))
+        line["sliding_window"] = window_table(args.steps, args.warmup, device, peak)
         cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
         rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",

@@ -94,6 +94,25 @@ FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *l
            const int32_t *key_lens, fa_stream_t stream);
 
 /*
+ * fa_fwd_window -- fa_fwd with a sliding (local) window on top of the causal
+ * and key_lens masks: key j is also masked for query i when
+ * j < i + (N_k - N_q) - window_left, so a row sees at most the window_left
+ * keys before its diagonal position plus that position (with causal), and
+ * never keys before the window (without causal, the window bounds keys from
+ * below only).  This is the local-attention mask among the mask variants that
+ * "FlashAttention：把注意力从公式写成数据流" (section "精度、掩码和边界情况")
+ * groups with causal and padding masks.  Tiles wholly before a query block's
+ * window are never loaded; partially covered tiles are masked per element.
+ *
+ *   window_left   >= 0 (window_left >= N_k gives the same result as fa_fwd).
+ *   other arguments, ownership and errors as fa_fwd; FA_ERR_INVALID_ARG for a
+ *   negative window_left.
+ */
+FA_API int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                  const int32_t *key_lens, int window_left, fa_stream_t stream);
+
+/*
  * fa_fwd_host_workspace_size -- bytes of device workspace fa_fwd_host needs
  * for this problem (room for Q, K, V, O, LSE and key_lens on the device,
  * each 256-byte aligned).  Returns 0 for invalid sizes.

@@ -87,6 +87,7 @@ struct FwdParams {
     int B, H, Nq, Nk;
     float scale_log2;           // scale * log2(e), > 0
     int causal;
+    int window_left;            // sliding window: keys before i+off-window_left are masked; < 0: none
     unsigned long long wait_limit;  // clock64 cycles per wait before giving up
     // split-KV mode only: each Q tile's K/V tiles are cut into num_splits
     // contiguous ranges, one CTA each, writing a partial result per range
@@ -242,6 +243,13 @@ __device__ __forceinline__ float chunk_max32(const float (&s)[kBlockN], int o) {
     return max3f(max3f(b0, b1, b2), a[9], a[10]);
 }
 
+// First key a query row may see: the sliding-window start (0 without a window).
+__device__ __forceinline__ int row_key_start(int row, int off, int window_left) {
+    if (window_left < 0) return 0;
+    const long long c = (long long)row + off - window_left;
+    return c < 0 ? 0 : (c > 0x7fffffffLL ? 0x7fffffff : (int)c);
+}
+
 // Number of keys (prefix length) a query row may see.
 __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causal) {
     if (!causal) return kl;
@@ -310,8 +318,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // split-KV mode this CTA takes tiles t0 .. t0+n_kv-1 of them.
     const int last_row = min(m0 + kBlockM - 1, p.Nq - 1);
     const int n_all = (row_key_limit(last_row, kl, off, p.causal) + kBlockN - 1) / kBlockN;
-    const int t0 = kSplit ? (int)((long long)split * n_all / n_split) : 0;
-    const int n_kv = kSplit ? (int)((long long)(split + 1) * n_all / n_split) - t0 : n_all;
+    // With a sliding window the first row's window start bounds the tiles from below.
+    const int t_lo = min(row_key_start(m0, off, p.window_left) / kBlockN, n_all);
+    const int n_span = n_all - t_lo;
+    const int t0 = t_lo + (kSplit ? (int)((long long)split * n_span / n_split) : 0);
+    const int n_kv = kSplit ? t_lo + (int)((long long)(split + 1) * n_span / n_split) - t0 : n_span;
 
     // ---- setup: barriers (producer lane 0), TMEM (MMA warp)
     if (warp == kProducerWarp && lane == 0) {
@@ -458,6 +469,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
         const int row = m0 + r;
         const int lim = row_key_limit(row, kl, off, p.causal);
+        const int lo = row_key_start(row, off, p.window_left);   // 0 without a window
         const float c = p.scale_log2;
         float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
         float lu = 0.f;            // the same sum before rounding (for the LSE)
@@ -491,11 +503,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             if (lane == 0) mbar_arrive(bar_s_free(j % C::kSBufs));
             const int kbase = (t0 + j) * kBlockN;
             // warp-uniform: the element mask runs only on tiles that cross a row's key limit
-            const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim);
+            const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim || kbase < lo);
             if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBlockN; ++i)
-                    if (kbase + i >= lim) s[i] = -INFINITY;
+                    if (kbase + i >= lim || kbase + i < lo) s[i] = -INFINITY;
             }
             const float mx = fmaxf(fmaxf(chunk_max32(s, 0), chunk_max32(s, 32)),
                                    fmaxf(chunk_max32(s, 64), chunk_max32(s, 96)));

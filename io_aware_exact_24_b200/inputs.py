@@ -45,10 +45,19 @@ class Workload:
     sigma: float = 1.0
     key_len_range: tuple[int, int] | None = None  # inclusive; None = no padding
     seed: int = 0
+    window_left: int = -1                          # sliding window (fa_fwd_window); -1 = none
 
     @property
     def flop(self) -> float:
-        """4*B*H*Nq*Nk*d, causal counted as exactly half."""
+        """4*B*H*Nq*Nk*d, causal counted as exactly half; with a sliding window,
+        4*B*H*d times the exact number of visible (query, key) pairs."""
+        if self.window_left >= 0:
+            i = np.arange(self.Nq, dtype=np.int64)
+            diag = i + (self.Nk - self.Nq)
+            hi = np.minimum(diag + 1, self.Nk) if self.causal else np.full_like(i, self.Nk)
+            lo = np.maximum(diag - self.window_left, 0)
+            pairs = int(np.maximum(hi - lo, 0).sum())
+            return 4.0 * self.B * self.H * self.d * pairs
         f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
         return f / 2.0 if self.causal else f
 
@@ -134,3 +143,11 @@ def make_inputs(w: Workload):
     if w.key_len_range is not None:
         kl = key_lengths(w.B, w.key_len_range[0], w.key_len_range[1], w.seed)
     return {"q": q, "k": k, "v": v, "key_lens": kl}
+
+# Sliding-window (local) causal attention for fa_fwd_window: each query sees the
+# 2048 keys before its position and itself.
+WINDOW_WORKLOADS = {
+    "window_16k_w2k_d128": Workload("window_16k_w2k_d128", 1, 16, 16384, 16384, 128, True,
+                                    float(np.float32(1 / math.sqrt(128))), 1.0, None, 8,
+                                    window_left=2048),
+}

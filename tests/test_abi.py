@@ -182,3 +182,32 @@ def test_splitkv_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert splitkv_call() == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- sliding window entry point
+
+def window_call(window_left=16, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Nq=8, Nk=8, d=64, scale=0.125, causal=1,
+             key_lens=None)
+    a.update(kw)
+    return binding.fa_fwd_window(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                                 a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                                 a["key_lens"], window_left, stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(window_left=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(window_left=-100, B=0), binding.FA_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(o=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(Nq=0), binding.FA_OK),
+])
+def test_window_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert window_call(**kw) == code
+
+
+def test_window_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert window_call(window_left=0) == binding.FA_ERR_NO_DEVICE

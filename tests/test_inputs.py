@@ -47,3 +47,12 @@ def test_workload_shapes():
     w = WORKLOADS["causal_8000_d128"]
     assert w.flop == 4 * 2 * 32 * 8000 * 8000 * 128 / 2
     assert WORKLOADS["long_16k_d64"].flop == 4 * 16 * 16384**2 * 64
+
+
+def test_window_flop_counts_visible_pairs():
+    from io_aware_exact_24_b200.inputs import Workload
+    for Nq, Nk, causal, W in ((9, 9, True, 3), (5, 12, True, 0), (12, 5, True, 2), (6, 10, False, 4)):
+        w = Workload("t", 2, 3, Nq, Nk, 8, causal, 0.1, window_left=W)
+        pairs = sum(1 for i in range(Nq) for j in range(Nk)
+                    if j >= i + Nk - Nq - W and (not causal or j <= i + Nk - Nq))
+        assert w.flop == 4.0 * 2 * 3 * 8 * pairs
