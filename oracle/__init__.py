@@ -66,6 +66,9 @@ def _load():
             lib.attn_ref_fp64_window.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                                  f32, i32, i64, vp, vp, vp]
             lib.attn_ref_fp64_window.restype = i32
+            lib.attn_ref_fp64_bias.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                               f32, i32, i64, vp, vp, vp, vp]
+            lib.attn_ref_fp64_bias.restype = i32
             lib.attn_ref_fp64_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
                                                i64, f32, i32, vp, i64, vp, vp]
             lib.attn_ref_fp64_rows.restype = i32
@@ -128,6 +131,23 @@ def attn_ref_window(q, k, v, scale, window_left, causal=False, key_lens=None):
                                       int(window_left), _ptr(o), _ptr(lse), None)
     if rc != 0:
         raise RuntimeError(f"attn_ref_fp64_window failed ({rc})")
+    return o, lse
+
+
+def attn_ref_bias(q, k, v, scale, slopes, causal=False, key_lens=None, window_left=-1):
+    """Plain definition with the additive positional bias -slopes[h]*|i + Nk - Nq - j|
+    (slopes: fp32 [H]) and optionally a sliding window.  Returns (O, LSE) in fp64."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    sl = np.ascontiguousarray(slopes, dtype=np.float32)
+    if sl.shape != (H,):
+        raise ValueError("slopes must be fp32 [H]")
+    o = np.empty((B, H, Nq, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    rc = _load().attn_ref_fp64_bias(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H, Nq, Nk,
+                                    d, float(np.float32(scale)), int(bool(causal)),
+                                    int(window_left), _ptr(sl), _ptr(o), _ptr(lse), None)
+    if rc != 0:
+        raise RuntimeError(f"attn_ref_fp64_bias failed ({rc})")
     return o, lse
 
 

@@ -27,6 +27,10 @@
  *     keys before its diagonal position plus that position.  This is the
  *     local-attention mask of the "mask variants" the second page's section
  *     "精度、掩码和边界情况" groups with causal and padding masks.
+ *   - additive positional bias (attn_ref_fp64_bias only): with per-head slopes
+ *     m_h, S_ij += -m_h * |i + (N_k - N_q) - j| on the visible entries (a
+ *     linear distance penalty from the row's diagonal position, the
+ *     "additive positional bias" mask variant).
  *
  * Nothing here is shared with the CUDA path.  Only tests/, the package's
  * graft entry smoke check and bench.py's CPU baseline may call it.
@@ -87,15 +91,17 @@ static int64_t row_start(int64_t i, int64_t Nq, int64_t Nk, int64_t W) {
  */
 static void one_row(const uint16_t *q_row, const uint16_t *k_head,
                     const uint16_t *v_head, int64_t Nk, int64_t d,
-                    double scale, int64_t lo, int64_t lim, double *s_row, double *p_row,
-                    double *o_row, double *lse_out) {
-    /* S_ij = scale * sum_c q_ic k_jc for valid j, -inf for masked j. */
+                    double scale, int64_t lo, int64_t lim, double slope, int64_t pos,
+                    double *s_row, double *p_row, double *o_row, double *lse_out) {
+    /* S_ij = scale * sum_c q_ic k_jc (- slope * |pos - j|) for valid j, -inf
+     * for masked j. */
     for (int64_t j = 0; j < Nk; ++j) {
         if (j >= lo && j < lim) {
             double dot = 0.0;
             for (int64_t c = 0; c < d; ++c)
                 dot += bf16_bits_to_f64(q_row[c]) * bf16_bits_to_f64(k_head[j * d + c]);
             s_row[j] = scale * dot;
+            if (slope != 0.0) s_row[j] -= slope * (double)llabs(pos - j);
         } else {
             s_row[j] = -INFINITY;
         }
@@ -136,10 +142,29 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
  * position, see the header comment; W < 0 means no window and gives exactly
  * attn_ref_fp64).  Arguments otherwise as attn_ref_fp64.
  */
+int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                       int64_t Nk, int64_t d, float scale, int causal,
+                       int64_t window_left, const float *slopes, double *o, double *lse,
+                       double *p_out);
+
 int attn_ref_fp64_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
                          int64_t Nk, int64_t d, float scale, int causal,
                          int64_t window_left, double *o, double *lse, double *p_out) {
+    return attn_ref_fp64_bias(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, window_left,
+                              NULL, o, lse, p_out);
+}
+
+/*
+ * Forward with a sliding window (window_left < 0: none) and an additive
+ * positional bias (slopes: fp32 [H], one slope per head, or NULL: none).
+ */
+int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                       int64_t Nk, int64_t d, float scale, int causal,
+                       int64_t window_left, const float *slopes, double *o, double *lse,
+                       double *p_out) {
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0) return -1;
     const double sc = (double)scale;
     const int64_t rows = B * H * Nq;
@@ -159,8 +184,9 @@ int attn_ref_fp64_window(const uint16_t *q, const uint16_t *k, const uint16_t *v
                 const int64_t b = bh / H;
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
                 const int64_t lo = row_start(i, Nq, Nk, window_left);
+                const double slope = slopes ? (double)slopes[bh % H] : 0.0;
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        lo, lim, s_row, p_row, o + r * d, lse + r);
+                        lo, lim, slope, i + (Nk - Nq), s_row, p_row, o + r * d, lse + r);
                 if (p_out) memcpy(p_out + r * Nk, p_row, sizeof(double) * (size_t)Nk);
             }
         }
@@ -210,7 +236,7 @@ int attn_ref_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const int64_t b = bh / H;
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        0, lim, s_row, p_row, o_rows + t * d, lse_rows + t);
+                        0, lim, 0.0, i + (Nk - Nq), s_row, p_row, o_rows + t * d, lse_rows + t);
             }
         }
         free(s_row);

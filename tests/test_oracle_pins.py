@@ -312,3 +312,67 @@ def test_wide_window_is_no_window(causal):
         assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
     o2, l2 = oracle.attn_ref_window(q, k, v, 0.2, -1, causal, kl)
     assert np.array_equal(o0, o2) and np.array_equal(l0, l2)
+
+
+# ---------------------------------------------------------------- additive positional bias
+
+def test_zero_slopes_are_no_bias():
+    q, k, v = _rand(2, 3, 9, 14, 8, 34)
+    kl = np.array([14, 6], np.int32)
+    for causal in (False, True):
+        o0, l0 = oracle.attn_ref(q, k, v, 0.2, causal, kl)
+        o1, l1 = oracle.attn_ref_bias(q, k, v, 0.2, np.zeros(3, np.float32), causal, kl)
+        assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_bias_with_zero_query_is_a_geometric_weighting():
+    # q = 0: scores are the bias alone, -m*(pos - j) for j <= pos (causal), so
+    # LSE = ln sum_{t=0}^{pos} e^{-m t} = ln((1 - e^{-m(pos+1)}) / (1 - e^{-m}))
+    # and O is the e^{-m(pos-j)}-weighted mean of the visible value rows
+    B, H, N, d = 1, 2, 13, 8
+    _, k, v = _rand(B, H, N, N, d, 35)
+    q = np.zeros((B, H, N, d), np.uint16)
+    slopes = np.array([0.5, 0.0625], np.float32)
+    o, lse = oracle.attn_ref_bias(q, k, v, 0.3, slopes, True, None)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    for h in range(H):
+        m = float(slopes[h])
+        for i in range(N):
+            closed = math.log((1 - math.exp(-m * (i + 1))) / (1 - math.exp(-m)))
+            assert abs(lse[0, h, i] - closed) <= 1e-12
+            w = np.exp(-m * (i - np.arange(i + 1)))
+            np.testing.assert_allclose(o[0, h, i], (w[:, None] * vf[0, h, :i + 1]).sum(0) / w.sum(),
+                                       rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,W", [(True, -1), (False, -1), (True, 5)])
+def test_bias_matches_torch_sdpa_with_an_additive_mask(causal, W):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+    B, H, Nq, Nk, d = 2, 2, 11, 17, 8
+    q, k, v = _rand(B, H, Nq, Nk, d, 36)
+    kl = np.array([17, 9], np.int32)
+    slopes = np.array([0.25, 0.03125], np.float32)
+    scale = 0.2
+    o, lse = oracle.attn_ref_bias(q, k, v, scale, slopes, causal, kl, W)
+    tq, tk, tv = (torch.from_numpy(bf16_bits_to_f32(x).astype(np.float64)) for x in (q, k, v))
+    i = np.arange(Nq)[:, None] + (Nk - Nq)
+    j = np.arange(Nk)[None, :]
+    bias = np.zeros((B, H, Nq, Nk))
+    for b in range(B):
+        vis = j < kl[b]
+        if causal:
+            vis = vis & (j <= i)
+        if W >= 0:
+            vis = vis & (j >= i - W)
+        for h in range(H):
+            bias[b, h] = np.where(vis, -float(slopes[h]) * np.abs(i - j), -np.inf)
+    tb = torch.from_numpy(bias)
+    ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=tb,
+                                         scale=float(np.float32(scale))).numpy()
+    ref_lse = torch.logsumexp(torch.einsum("bhid,bhjd->bhij", tq, tk) * float(np.float32(scale))
+                              + tb, dim=-1).numpy()
+    has = np.isfinite(ref_lse)
+    np.testing.assert_allclose(o[has], ref[has], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[has], ref_lse[has], rtol=0, atol=1e-12)
+    assert np.all(np.isneginf(lse[~has]))
