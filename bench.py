@@ -177,26 +177,35 @@ def time_device(w, x, steps, warmup, device, rank, world, clocks=None):
 
 
 def time_window(w, x, steps, warmup, device):
-    """Mean per-call device time (ms) of fa_fwd_window, L2 flushed between calls."""
+    """Mean per-call device time (ms) of fa_fwd_window / fa_fwd_bias, L2 flushed between calls."""
     import torch
-    from io_aware_exact_24_b200 import fa_fwd_window
+    from io_aware_exact_24_b200 import fa_fwd_bias, fa_fwd_window
+    from io_aware_exact_24_b200.inputs import alibi_slopes
     q, k, v, kl = upload(x, device)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+    slopes = torch.from_numpy(alibi_slopes(w.H)).to(device) if w.alibi else None
+
+    def launch():
+        if w.alibi:
+            fa_fwd_bias(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
+                        slopes, w.window_left, stream)
+        else:
+            fa_fwd_window(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
+                          w.window_left, stream)
+
     for _ in range(warmup):
         flush.zero_()
-        fa_fwd_window(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
-                      w.window_left, stream)
+        launch()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     for st, en in ev:
         flush.zero_()
         st.record(stream)
-        fa_fwd_window(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl,
-                      w.window_left, stream)
+        launch()
         en.record(stream)
     torch.cuda.synchronize()
     per = [st.elapsed_time(en) for st, en in ev]
@@ -205,17 +214,19 @@ def time_window(w, x, steps, warmup, device):
 
 
 def window_table(steps, warmup, device, peak_tflops):
-    """Sliding-window forward: TFLOP/s on the visible (query, key) pairs only."""
+    """Mask variants: TFLOP/s (a window counts the visible query-key pairs only)."""
     out = {}
     for name, w in WINDOW_WORKLOADS.items():
         x = make_inputs(w)
         ms = time_window(w, x, steps, warmup, device)
         tf = w.flop / (ms / 1000.0) / 1e12
-        out[name] = {"entry": "fa_fwd_window", "window_left": w.window_left, "ms": ms,
+        out[name] = {"entry": "fa_fwd_bias" if w.alibi else "fa_fwd_window",
+                     "window_left": w.window_left, "alibi": w.alibi, "ms": ms,
                      "tflops": tf, "roofline": {"bound": "tensor", "achieved": tf,
                                                 "peak": peak_tflops, "unit": "TFLOP/s",
                                                 "frac": tf / peak_tflops},
-                     "flop": "4*B*H*d*(visible query-key pairs)",
+                     "flop": ("4*B*H*d*(visible query-key pairs)" if w.window_left >= 0
+                              else "4*B*H*Nq*Nk*d, causal halved"),
                      "config": config_of(w, "flushed between timed launches", "single GPU")}
         del x
     return out

@@ -113,6 +113,26 @@ FA_API int fa_fwd_window(const void *q, const void *k, const void *v, void *o, f
                   const int32_t *key_lens, int window_left, fa_stream_t stream);
 
 /*
+ * fa_fwd_bias -- fa_fwd with an additive positional bias (and, optionally, the
+ * sliding window of fa_fwd_window): before the softmax every visible score
+ * gets -slopes[h] * |i + (N_k - N_q) - j|, a linear penalty on the distance
+ * from the row's diagonal position (the "additive positional bias" mask
+ * variant of "FlashAttention：把注意力从公式写成数据流", section
+ * "精度、掩码和边界情况"; with the usual per-head slopes this is the ALiBi
+ * bias).  The LSE includes the bias.
+ *
+ *   slopes        device fp32 [H], 4-byte aligned, non-NULL (finite; >= 0 for
+ *                 the usual decaying bias, any sign is computed as given).
+ *   window_left   < 0: no window; >= 0: as fa_fwd_window.
+ *   other arguments, ownership and errors as fa_fwd; FA_ERR_INVALID_ARG for
+ *   NULL slopes, FA_ERR_MISALIGNED for unaligned slopes.
+ */
+FA_API int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                const int32_t *key_lens, const float *slopes, int window_left,
+                fa_stream_t stream);
+
+/*
  * fa_fwd_host_workspace_size -- bytes of device workspace fa_fwd_host needs
  * for this problem (room for Q, K, V, O, LSE and key_lens on the device,
  * each 256-byte aligned).  Returns 0 for invalid sizes.

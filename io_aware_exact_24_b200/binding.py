@@ -58,6 +58,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                           vp, i32, vp]
             lib.fa_fwd_window.restype = i32
+            lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
+                                        vp, vp, i32, vp]
+            lib.fa_fwd_bias.restype = i32
             lib.fa_fwd_host_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
             lib.fa_fwd_host_workspace_size.restype = sz
             lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
@@ -141,6 +144,18 @@ def fa_fwd_window(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, w
                                       _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_window")
+    return st
+
+
+def fa_fwd_bias(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, slopes,
+                window_left=-1, stream=None, check=True) -> int:
+    """``fa_fwd_bias`` of include/fa.h: forward with the additive positional bias."""
+    st = load_library().fa_fwd_bias(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                    int(B), int(H), int(N_q), int(N_k), int(d), float(scale),
+                                    int(bool(causal)), _addr(key_lens), _addr(slopes),
+                                    int(window_left), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_bias")
     return st
 
 

@@ -139,7 +139,7 @@ struct SplitParts {
 template <int D>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
            float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr},
-           int window_left = -1) {
+           int window_left = -1, const float* slopes = nullptr) {
     CUtensorMap tq, tk, tv, to;
     // With no keys the K/V maps are never read; give them a valid 1-row shape.
     const void* kp = N_k > 0 ? k : q;
@@ -161,6 +161,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.window_left = window_left;
+    p.slopes = slopes;
     p.wait_limit = kWaitLimitCycles;
     p.num_splits = sp.num_splits > 0 ? sp.num_splits : 1;
     p.o_part = sp.o_part;
@@ -407,6 +408,32 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
     const SplitParts none{0, nullptr, nullptr};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
+}
+
+int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
+                int d, float scale, int causal, const int32_t* key_lens, const float* slopes, int window_left,
+                fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (empty) return FA_OK;
+    if (slopes == nullptr) return FA_ERR_INVALID_ARG;
+    if (!aligned(slopes, 4)) return FA_ERR_MISALIGNED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const SplitParts none{0, nullptr, nullptr};
+    const int wl = window_left < 0 ? -1 : window_left;
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
 }
 
 size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has_key_lens) {

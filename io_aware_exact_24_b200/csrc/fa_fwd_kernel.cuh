@@ -88,6 +88,7 @@ struct FwdParams {
     float scale_log2;           // scale * log2(e), > 0
     int causal;
     int window_left;            // sliding window: keys before i+off-window_left are masked; < 0: none
+    const float* slopes;        // [H] additive positional bias -slopes[h]*|i+off-j|, or nullptr
     unsigned long long wait_limit;  // clock64 cycles per wait before giving up
     // split-KV mode only: each Q tile's K/V tiles are cut into num_splits
     // contiguous ranges, one CTA each, writing a partial result per range
@@ -470,6 +471,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int row = m0 + r;
         const int lim = row_key_limit(row, kl, off, p.causal);
         const int lo = row_key_start(row, off, p.window_left);   // 0 without a window
+        // additive positional bias, in log2 units per unit of distance (warp-uniform switch)
+        const bool has_bias = p.slopes != nullptr;
+        const float alpha = has_bias ? p.slopes[h] * 1.4426950408889634f : 0.f;
         const float c = p.scale_log2;
         float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
         float lu = 0.f;            // the same sum before rounding (for the LSE)
@@ -504,6 +508,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const int kbase = (t0 + j) * kBlockN;
             // warp-uniform: the element mask runs only on tiles that cross a row's key limit
             const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim || kbase < lo);
+            if (has_bias) {
+                // t_i = s_i * c - alpha * |row + off - (kbase + i)|; from here on the
+                // scores are in log2 units already (scale factor 1)
+                const float d0 = (float)(row + off - kbase);
+#pragma unroll
+                for (int i = 0; i < kBlockN; ++i) s[i] = fmaf(s[i], c, -alpha * fabsf(d0 - (float)i));
+            }
+            const float cs = has_bias ? 1.f : c;
             if (masked) {
 #pragma unroll
                 for (int i = 0; i < kBlockN; ++i)
@@ -522,7 +534,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
                 m_prev = mref[(g ^ 1) * kBlockM + r];
             }
-            const float t_max = mx * c;   // c > 0, so -inf stays -inf
+            const float t_max = mx * cs;  // cs > 0, so -inf stays -inf
             const float m_cur = (t_max > m_prev + kRescaleThreshold) ? t_max : m_prev;
             if (j + 1 < n_kv) {
                 mref[g * kBlockM + r] = m_cur;
@@ -548,11 +560,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             float2 lu2 = make_float2(0.f, 0.f);
             const uint32_t taddr_p = tmem + lane_off + C::col_p(pb);
             if (masked) {
-                exp_store_half<0, 0>(s, c, mu, taddr_p, lu2);
-                exp_store_half<0, 1>(s, c, mu, taddr_p, lu2);
+                exp_store_half<0, 0>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<0, 1>(s, cs, mu, taddr_p, lu2);
             } else {
-                exp_store_half<C::kEmuPairs, 0>(s, c, mu, taddr_p, lu2);
-                exp_store_half<C::kEmuPairs, 1>(s, c, mu, taddr_p, lu2);
+                exp_store_half<C::kEmuPairs, 0>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<C::kEmuPairs, 1>(s, cs, mu, taddr_p, lu2);
             }
             lu += lu2.x + lu2.y;
             // O holds tiles < j relative to m_prev.  Only when some row of this

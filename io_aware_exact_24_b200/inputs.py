@@ -46,6 +46,7 @@ class Workload:
     key_len_range: tuple[int, int] | None = None  # inclusive; None = no padding
     seed: int = 0
     window_left: int = -1                          # sliding window (fa_fwd_window); -1 = none
+    alibi: bool = False                            # additive positional bias with alibi_slopes(H)
 
     @property
     def flop(self) -> float:
@@ -144,10 +145,19 @@ def make_inputs(w: Workload):
         kl = key_lengths(w.B, w.key_len_range[0], w.key_len_range[1], w.seed)
     return {"q": q, "k": k, "v": v, "key_lens": kl}
 
-# Sliding-window (local) causal attention for fa_fwd_window: each query sees the
-# 2048 keys before its position and itself.
+def alibi_slopes(H: int) -> np.ndarray:
+    """The usual geometric per-head bias slopes 2^(-8(h+1)/H), fp32 [H]."""
+    return (2.0 ** (-8.0 * (np.arange(H) + 1) / H)).astype(np.float32)
+
+
+# Mask variants: sliding-window (local) causal attention for fa_fwd_window, each
+# query seeing the 2048 keys before its position and itself; and the
+# causal_8000_d128 shape with the additive positional bias (fa_fwd_bias).
 WINDOW_WORKLOADS = {
     "window_16k_w2k_d128": Workload("window_16k_w2k_d128", 1, 16, 16384, 16384, 128, True,
                                     float(np.float32(1 / math.sqrt(128))), 1.0, None, 8,
                                     window_left=2048),
+    "alibi_causal_8000_d128": Workload("alibi_causal_8000_d128", 2, 32, 8000, 8000, 128, True,
+                                       float(np.float32(1 / math.sqrt(128))), 0.5, None, 5,
+                                       alibi=True),
 }

@@ -211,3 +211,32 @@ def test_window_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert window_call(window_left=0) == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- additive bias entry point
+
+def bias_call(slopes=P, window_left=-1, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, Nq=8, Nk=8, d=64, scale=0.125, causal=1,
+             key_lens=None)
+    a.update(kw)
+    return binding.fa_fwd_bias(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                               a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], a["key_lens"],
+                               slopes, window_left, stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(slopes=None), binding.FA_ERR_INVALID_ARG),
+    (dict(slopes=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=-1.0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0, slopes=None), binding.FA_OK),
+])
+def test_bias_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert bias_call(**kw) == code
+
+
+def test_bias_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert bias_call() == binding.FA_ERR_NO_DEVICE
