@@ -232,6 +232,56 @@ def window_table(steps, warmup, device, peak_tflops):
     return out
 
 
+def varlen_table(steps, warmup, device, peak_tflops):
+    """Packed variable-length batch with the BERT-shaped lengths of bert_padded_512
+    (each sequence's queries and keys = its key length), against the padded
+    fa_fwd run of the same batch.  TFLOP/s on the real (unpadded) work."""
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd_varlen
+    w = WORKLOADS["bert_padded_512"]
+    x = make_inputs(w)
+    lens = x["key_lens"].astype(np.int64)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    pack = lambda a: np.ascontiguousarray(np.concatenate(
+        [a[b, :, :lens[b]].transpose(1, 0, 2) for b in range(w.B)], axis=0))
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    q, k, v = dev(pack(x["q"])), dev(pack(x["k"])), dev(pack(x["v"]))
+    o = torch.empty_like(q)
+    lse = torch.empty((T, w.H), dtype=torch.float32, device=device)
+    tcu = torch.from_numpy(cu).to(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    maxq = int(lens.max())
+
+    def launch():
+        fa_fwd_varlen(q, k, v, o, lse, tcu, tcu, w.B, w.H, T, T, maxq, w.d, w.scale, False, stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for st, en in ev:
+        flush.zero_()
+        st.record(stream)
+        launch()
+        en.record(stream)
+    torch.cuda.synchronize()
+    ms = float(np.mean([st.elapsed_time(en) for st, en in ev]))
+    ms_pad, _, _ = time_device(w, x, steps, warmup, device, 0, 1)
+    flop = 4.0 * w.H * w.d * float((lens * lens).sum())
+    tf = flop / (ms / 1000.0) / 1e12
+    return {"varlen_bert_d64": {"entry": "fa_fwd_varlen", "B": w.B, "H": w.H, "d": w.d,
+                                "total_tokens": T, "max_seqlen": maxq, "ms": ms, "tflops": tf,
+                                "flop": "4*H*d*sum_b len_b^2 (no padding)",
+                                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tflops,
+                                             "unit": "TFLOP/s", "frac": tf / peak_tflops},
+                                "padded_fa_fwd_ms": ms_pad,
+                                "config": "bert_padded_512 inputs, each sequence packed to its key length"}}
+
+
 def time_splitkv(w, x, steps, warmup, device, num_splits=None):
     """Mean per-call device time (ms) of fa_fwd_splitkv (partials + merge), L2 flushed between calls."""
     import torch
@@ -490,6 +540,7 @@ def main():
         line["splitkv_decode"] = decode_table(args.steps, args.warmup, device,
                                               float(peaks["hbm_gbs"]))
         line["sliding_window"] = window_table(args.steps, args.warmup, device, peak)
+        line["varlen"] = varlen_table(args.steps, args.warmup, device, peak)
         cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
         rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",

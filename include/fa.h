@@ -133,6 +133,40 @@ FA_API int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, flo
                 fa_stream_t stream);
 
 /*
+ * fa_fwd_varlen -- attention over a batch of sequences of different lengths
+ * packed back to back without padding (the packed variable-length batches of
+ * the mask variants, "FlashAttention：把注意力从公式写成数据流", section
+ * "精度、掩码和边界情况": ragged tails and no work on padding).  Sequence b
+ * is an independent problem: its queries are tokens cu_seqlens_q[b] ..
+ * cu_seqlens_q[b+1]-1, its keys tokens cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1,
+ * with the causal alignment of fa_fwd applied to its own lengths.
+ *
+ *   q           device bf16 [total_q, H, d] (token-major), 16-byte aligned.
+ *   k, v        device bf16 [total_k, H, d], 16-byte aligned (may be NULL when
+ *               total_k == 0).
+ *   o           device bf16 [total_q, H, d], 16-byte aligned; rows of every
+ *               sequence written, nothing else.
+ *   lse         device fp32 [total_q, H], 4-byte aligned.
+ *   cu_seqlens_q, cu_seqlens_k   device int32 [B+1], 4-byte aligned,
+ *               non-decreasing, starting at 0 and ending at total_q / total_k.
+ *               A sequence whose offsets fall outside [0, total] is treated as
+ *               empty (nothing written for it).
+ *   max_seqlen_q  at least every query length (sizes the grid; longer
+ *               sequences are cut at it).
+ *   scale, causal, d, stream   as for fa_fwd (no key_lens: lengths come from
+ *               cu_seqlens_k).
+ *
+ * Returns FA_OK once enqueued, FA_ERR_INVALID_ARG / FA_ERR_MISALIGNED /
+ * FA_ERR_UNSUPPORTED for bad arguments (checked before any CUDA call),
+ * FA_ERR_NO_DEVICE or FA_ERR_CUDA otherwise.  B, H, total_q or max_seqlen_q
+ * equal to 0 is a no-op.
+ */
+FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int B, int H,
+                  int total_q, int total_k, int max_seqlen_q, int d, float scale, int causal,
+                  fa_stream_t stream);
+
+/*
  * fa_fwd_host_workspace_size -- bytes of device workspace fa_fwd_host needs
  * for this problem (room for Q, K, V, O, LSE and key_lens on the device,
  * each 256-byte aligned).  Returns 0 for invalid sizes.

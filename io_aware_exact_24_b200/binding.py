@@ -61,6 +61,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                         vp, vp, i32, vp]
             lib.fa_fwd_bias.restype = i32
+            lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                          f32, i32, vp]
+            lib.fa_fwd_varlen.restype = i32
             lib.fa_fwd_host_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
             lib.fa_fwd_host_workspace_size.restype = sz
             lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
@@ -156,6 +159,18 @@ def fa_fwd_bias(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, slo
                                     int(window_left), _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_bias")
+    return st
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k,
+                  max_seqlen_q, d, scale, causal=False, stream=None, check=True) -> int:
+    """``fa_fwd_varlen`` of include/fa.h: packed variable-length batches."""
+    st = load_library().fa_fwd_varlen(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                      _addr(cu_seqlens_q), _addr(cu_seqlens_k), int(B), int(H),
+                                      int(total_q), int(total_k), int(max_seqlen_q), int(d),
+                                      float(scale), int(bool(causal)), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
     return st
 
 

@@ -81,6 +81,12 @@ int prepare_device(int dev) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
         if (e != cudaSuccess) {
             st.status = cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
             return;
@@ -136,6 +142,56 @@ struct SplitParts {
     float* lse_part;
 };
 
+// Packed [T, H, d] bf16 viewed as (d, H, T, 1), box 64 x 1 x 128 x 1: the same
+// 128-token x 64-column shared-memory tile as the dense map, for one head.
+bool encode_thd(CUtensorMap* map, const void* ptr, int T, int H, int d) {
+    EncodeTiledFn enc = encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)fa::kBlockM, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_q,
+                  const int32_t* cu_k, int B, int H, int T_q, int T_k, int max_q, float scale, int causal,
+                  cudaStream_t stream) {
+    CUtensorMap tq, tk, tv;
+    const void* kp = T_k > 0 ? k : q;
+    const void* vp = T_k > 0 ? v : q;
+    const int tk_map = T_k > 0 ? T_k : 1;
+    if (!encode_thd(&tq, q, T_q, H, D) || !encode_thd(&tk, kp, tk_map, H, D) || !encode_thd(&tv, vp, tk_map, H, D)) {
+        snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
+        return FA_ERR_CUDA;
+    }
+    fa::FwdParams p{};
+    p.lse = lse;
+    p.key_lens = nullptr;
+    p.B = B;
+    p.H = H;
+    p.Nq = T_q;
+    p.Nk = T_k;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.window_left = -1;
+    p.slopes = nullptr;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.o_packed = reinterpret_cast<__nv_bfloat16*>(o);
+    p.wait_limit = kWaitLimitCycles;
+    p.num_splits = 1;
+    dim3 grid((unsigned)((max_q + fa::kBlockM - 1) / fa::kBlockM), (unsigned)H, (unsigned)B);
+    // the O map is never used in this mode; any valid map will do
+    fa::fa_fwd_sm100_kernel<D, false, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv,
+                                                                                                     tq, p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (packed variable-length)", e);
+}
+
 template <int D>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
            float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr},
@@ -151,7 +207,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
         return FA_ERR_CUDA;
     }
-    fa::FwdParams p;
+    fa::FwdParams p{};
     p.lse = lse;
     p.key_lens = key_lens;
     p.B = B;
@@ -434,6 +490,43 @@ int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse
     const int wl = window_left < 0 ? -1 : window_left;
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                  const int32_t* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q, int d,
+                  float scale, int causal, fa_stream_t stream) {
+    if (B < 0 || H < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (!(scale * 1.4426950408889634f > 0.f) || !std::isfinite(scale * 1.4426950408889634f))
+        return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || total_q == 0 || max_seqlen_q == 0) return FA_OK;
+    if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;
+    if ((unsigned long long)total_q * H * d * 2 >= (1ull << 40) || (unsigned long long)total_k * H * d * 2 >= (1ull << 40))
+        return FA_ERR_UNSUPPORTED;
+    if (q == nullptr || o == nullptr || lse == nullptr || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)
+        return FA_ERR_INVALID_ARG;
+    if (total_k > 0 && (k == nullptr || v == nullptr)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(cu_seqlens_q, 4) ||
+        !aligned(cu_seqlens_k, 4))
+        return FA_ERR_MISALIGNED;
+    if (total_k > 0 && (!aligned(k, 16) || !aligned(v, 16))) return FA_ERR_MISALIGNED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    int st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return launch_varlen<64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q,
+                                 scale, causal, s);
+    return launch_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q,
+                              scale, causal, s);
 }
 
 size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has_key_lens) {

@@ -89,6 +89,12 @@ struct FwdParams {
     int causal;
     int window_left;            // sliding window: keys before i+off-window_left are masked; < 0: none
     const float* slopes;        // [H] additive positional bias -slopes[h]*|i+off-j|, or nullptr
+    // packed variable-length mode only: sequence b holds query tokens
+    // cu_q[b] .. cu_q[b+1]-1 and key tokens cu_k[b] .. cu_k[b+1]-1; Nq / Nk
+    // are then the token totals, Q/O are [Nq, H, D], K/V [Nk, H, D], LSE [Nq, H]
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    __nv_bfloat16* o_packed;    // O of the packed mode (written with plain stores)
     unsigned long long wait_limit;  // clock64 cycles per wait before giving up
     // split-KV mode only: each Q tile's K/V tiles are cut into num_splits
     // contiguous ranges, one CTA each, writing a partial result per range
@@ -265,7 +271,9 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
 // Memory-Efficient Exact Attention with IO-Awareness", its note on the decode
 // case): partial (O, LSE) for one contiguous range of K/V tiles, merged by
 // fa_splitkv_combine_kernel.
-template <int D, bool kSplit = false>
+// kVarlen = true: packed variable-length batches (FwdParams::cu_q / cu_k);
+// the TMA maps then view [tokens, H, D] as (D, H, tokens, 1).
+template <int D, bool kSplit = false, bool kVarlen = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -309,15 +317,40 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int m0 = m_blk * kBlockM;
-    int kl = p.Nk;
+    // this (b, h) problem's sizes, and where its rows start in the tensors
+    int Nq_b = p.Nq, Nk_b = p.Nk, q_base = 0, k_base = 0;
+    if constexpr (kVarlen) {
+        q_base = p.cu_q[b];
+        k_base = p.cu_k[b];
+        Nq_b = p.cu_q[b + 1] - q_base;
+        Nk_b = p.cu_k[b + 1] - k_base;
+        // offsets outside the packed tensors make the sequence empty (nothing is written)
+        if (q_base < 0 || Nq_b < 0 || q_base > p.Nq - Nq_b) Nq_b = 0;
+        if (k_base < 0 || Nk_b < 0 || k_base > p.Nk - Nk_b) Nk_b = 0;
+        if (m0 >= Nq_b) return;   // the whole CTA, before any setup
+    }
+    int kl = Nk_b;
     if (p.key_lens != nullptr) {
         kl = p.key_lens[b];
-        kl = kl < 0 ? 0 : (kl > p.Nk ? p.Nk : kl);
+        kl = kl < 0 ? 0 : (kl > Nk_b ? Nk_b : kl);
     }
-    const int off = p.Nk - p.Nq;  // causal diagonal offset (bottom-right aligned)
+    const int off = Nk_b - Nq_b;  // causal diagonal offset (bottom-right aligned)
+    // TMA coordinates of a 128-row tile starting at row `r0` of this problem:
+    // (column, row, head, batch) dense, (column, head, token, 0) packed
+    auto tile_coords = [&](int base_tok, int r0, int& c1, int& c2, int& c3) {
+        if constexpr (kVarlen) {
+            c1 = h;
+            c2 = base_tok + r0;
+            c3 = 0;
+        } else {
+            c1 = r0;
+            c2 = h;
+            c3 = b;
+        }
+    };
     // K/V tiles this Q tile must visit: enough for its last real row; in
     // split-KV mode this CTA takes tiles t0 .. t0+n_kv-1 of them.
-    const int last_row = min(m0 + kBlockM - 1, p.Nq - 1);
+    const int last_row = min(m0 + kBlockM - 1, Nq_b - 1);
     const int n_all = (row_key_limit(last_row, kl, off, p.causal) + kBlockN - 1) / kBlockN;
     // With a sliding window the first row's window start bounds the tiles from below.
     const int t_lo = min(row_key_start(m0, off, p.window_left) / kBlockN, n_all);
@@ -379,8 +412,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const uint64_t pol_kv = policy_evict_last();
             if (rg == 0) {
                 mbar_arrive_expect_tx(bar_q_full, (uint32_t)C::kTileBytes);
+                int qc1, qc2, qc3;
+                tile_coords(q_base, m0, qc1, qc2, qc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, m0, h, b,
+                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, qc1, qc2, qc3,
                                 policy_evict_first());
             }
             bool ok = true;
@@ -391,9 +426,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 ok = wait_bounded(bar_empty(rg, s), (round & 1u) ^ 1u, abort_flag, p.wait_limit);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_full(rg, s), (uint32_t)C::kTileBytes);
+                int kc1, kc2, kc3;
+                tile_coords(k_base, (t0 + j) * kBlockN, kc1, kc2, kc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64,
-                                (t0 + j) * kBlockN, h, b, pol_kv);
+                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64, kc1, kc2,
+                                kc3, pol_kv);
             }
             if (!ok) {
                 // wind down: let every copy still in flight (at most one per
@@ -651,7 +688,26 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) u[i] = 0u;
                 }
-                if constexpr (kSplit) {
+                if constexpr (kVarlen) {
+                    // packed O: plain 16-byte stores of this row's chunk (a TMA
+                    // store would also write rows of the next sequence)
+                    if (row < Nq_b) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            p.o_packed + ((size_t)(q_base + row) * p.H + h) * D + col0);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            uint4 w4;
+                            w4.x = pack_bf16x2(__uint_as_float(u[8 * v4]) * inv_l, __uint_as_float(u[8 * v4 + 1]) * inv_l);
+                            w4.y = pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * inv_l,
+                                               __uint_as_float(u[8 * v4 + 3]) * inv_l);
+                            w4.z = pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * inv_l,
+                                               __uint_as_float(u[8 * v4 + 5]) * inv_l);
+                            w4.w = pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * inv_l,
+                                               __uint_as_float(u[8 * v4 + 7]) * inv_l);
+                            dst[v4] = w4;
+                        }
+                    }
+                } else if constexpr (kSplit) {
                     // partial O of this K/V range, fp32, straight to global memory
                     if (row < p.Nq) {
                         float4* dst = reinterpret_cast<float4*>(
@@ -680,9 +736,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                 }
             }
-            if (g == 0 && row < p.Nq) {
+            if (g == 0 && row < Nq_b) {
                 const float lse = (lu_row > 0.f) ? (m_fin + lg2_approx(lu_row)) * 0.69314718055994531f : -INFINITY;
-                if constexpr (kSplit)
+                if constexpr (kVarlen)
+                    p.lse[(size_t)(q_base + row) * p.H + h] = lse;
+                else if constexpr (kSplit)
                     p.lse_part[(((size_t)split * p.B + b) * p.H + h) * (size_t)p.Nq + row] = lse;
                 else
                     p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
@@ -690,7 +748,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
         fence_proxy_async_smem();
         const bool any_bad = named_bar_or(kBarSoftmaxAll, kSoftmaxWarps * 32, !good);
-        if (!kSplit && !any_bad && threadIdx.x == 0) {
+        if (!kSplit && !kVarlen && !any_bad && threadIdx.x == 0) {
             for (int bx = 0; bx < C::kBoxes; ++bx)
                 tma_store_4d(&tm_o, q_tile + bx * kSwizzleBoxBytes, bx * 64, m0, h, b);
             bulk_commit_group();

@@ -151,6 +151,29 @@ def attn_ref_bias(q, k, v, scale, slopes, causal=False, key_lens=None, window_le
     return o, lse
 
 
+def attn_ref_varlen(q, k, v, cu_q, cu_k, scale, causal=False):
+    """Packed variable-length batches: q [Tq,H,d], k/v [Tk,H,d] bf16 bits, cu_q/cu_k
+    int [B+1].  Each sequence is an independent problem, evaluated with attn_ref on
+    its own slice.  Returns (O fp64 [Tq,H,d], LSE fp64 [Tq,H])."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    Tq, H, d = q.shape
+    o = np.zeros((Tq, H, d), np.float64)
+    lse = np.full((Tq, H), -np.inf, np.float64)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 <= q0:
+            continue
+        qb = q[q0:q1].transpose(1, 0, 2)[None]
+        kb = k[k0:k1].transpose(1, 0, 2)[None]
+        vb = v[k0:k1].transpose(1, 0, 2)[None]
+        ob, lb = attn_ref(qb, kb, vb, scale, causal, None)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[q0:q1] = lb[0].T
+    return o, lse
+
+
 def attn_ref_rows(q, k, v, scale, row_ids, causal=False, key_lens=None):
     """Definition on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n])."""
     q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)

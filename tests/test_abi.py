@@ -240,3 +240,39 @@ def test_bias_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert bias_call() == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- packed variable-length entry point
+
+def varlen_call(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cu_q=P, cu_k=P, B=2, H=2, Tq=100, Tk=100, maxq=64, d=64,
+             scale=0.125, causal=1)
+    a.update(kw)
+    return binding.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu_q"], a["cu_k"],
+                                 a["B"], a["H"], a["Tq"], a["Tk"], a["maxq"], a["d"], a["scale"],
+                                 a["causal"], stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu_q=None), binding.FA_ERR_INVALID_ARG),
+    (dict(cu_k=None), binding.FA_ERR_INVALID_ARG),
+    (dict(cu_q=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(q=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(Tq=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(maxq=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(k=None), binding.FA_ERR_INVALID_ARG),
+    (dict(Tq=0), binding.FA_OK),
+    (dict(maxq=0), binding.FA_OK),
+    (dict(B=0, q=None, cu_q=None), binding.FA_OK),
+])
+def test_varlen_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert varlen_call(**kw) == code
+
+
+def test_varlen_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert varlen_call() == binding.FA_ERR_NO_DEVICE

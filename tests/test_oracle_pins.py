@@ -376,3 +376,15 @@ def test_bias_matches_torch_sdpa_with_an_additive_mask(causal, W):
     np.testing.assert_allclose(o[has], ref[has], rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse[has], ref_lse[has], rtol=0, atol=1e-12)
     assert np.all(np.isneginf(lse[~has]))
+
+
+def test_varlen_of_equal_lengths_is_the_dense_problem():
+    # packing B equal-length sequences token-major is a relayout of the dense batch
+    B, H, N, d = 3, 2, 9, 8
+    q, k, v = _rand(B, H, N, N, d, 37)
+    o, lse = oracle.attn_ref(q, k, v, 0.3, True, None)
+    pack = lambda x: x.transpose(0, 2, 1, 3).reshape(B * N, H, d)
+    cu = np.arange(B + 1) * N
+    ov, lv = oracle.attn_ref_varlen(pack(q), pack(k), pack(v), cu, cu, 0.3, True)
+    assert np.array_equal(ov, o.transpose(0, 2, 1, 3).reshape(B * N, H, d))
+    assert np.array_equal(lv, lse.transpose(0, 2, 1).reshape(B * N, H))
