@@ -28,6 +28,14 @@ int cuda_fail(const char* what, cudaError_t e) {
     return FA_ERR_CUDA;
 }
 constexpr unsigned long long kWaitLimitCycles = 1ull << 31;  // ~1 s at B200 clocks
+#ifndef FA_HEAD_GROUP_MB
+#define FA_HEAD_GROUP_MB 48
+#endif
+// share of the 126 MB L2 that the K/V of the (b, h) problems in flight may take
+constexpr long long kHeadGroupL2Bytes = (long long)FA_HEAD_GROUP_MB << 20;
+// below this many query blocks per (b, h) the per-CTA fixed cost dominates and
+// the plain order measured faster (GPT-2-sized causal problems, N = 1024)
+constexpr unsigned kHeadGroupMinBlocks = 32;
 constexpr int kMaxDevices = 64;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -224,6 +232,14 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.lse_part = sp.lse_part;
     const int rows_per_cta = fa::kBlockM;
     const unsigned num_m = (unsigned)((N_q + rows_per_cta - 1) / rows_per_cta);
+    if (sp.num_splits <= 0 && causal && num_m >= kHeadGroupMinBlocks) {
+        // causal blocks differ in cost: order the CTAs heaviest first inside groups
+        // of (b, h) problems whose K and V together fit in a share of the L2
+        const long long kv_head = 4LL * N_k * D;
+        long long hg = kHeadGroupL2Bytes / (kv_head > 0 ? kv_head : 1);
+        const long long hb = (long long)H * B;
+        p.head_group = (int)(hg < 1 ? 1 : (hg > hb ? hb : hg));
+    }
     if (sp.num_splits <= 0) {
         dim3 grid(num_m, (unsigned)H, (unsigned)B);
         fa::fa_fwd_sm100_kernel<D, false><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);

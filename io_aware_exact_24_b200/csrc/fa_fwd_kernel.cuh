@@ -101,6 +101,9 @@ struct FwdParams {
     int num_splits;
     float* o_part;              // [num_splits, B, H, Nq, D] fp32, O of the range / its own l
     float* lse_part;            // [num_splits, B, H, Nq] fp32, LSE of the range (-inf if empty)
+    // dense single-pass mode: > 1 reorders the CTAs' work (see the kernel); 0 or 1 keeps
+    // blockIdx = (query block, h, b)
+    int head_group;
 };
 
 template <int D>
@@ -311,11 +314,30 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ---- work item: (b, h, 128-row block[, K/V range]); heavy causal blocks launch first
     const int n_split = kSplit ? p.num_splits : 1;
     const int split = kSplit ? (int)blockIdx.x % n_split : 0;
-    const int blk = kSplit ? (int)blockIdx.x / n_split : (int)blockIdx.x;
+    int blk = kSplit ? (int)blockIdx.x / n_split : (int)blockIdx.x;
     const int num_m = (int)gridDim.x / n_split;
+    int h = blockIdx.y;
+    int b = blockIdx.z;
+    if constexpr (!kSplit && !kVarlen) {
+        if (p.head_group > 1) {
+            // CTAs start in linear order.  Walk the (b, h) problems in groups of
+            // head_group, and inside a group take every problem's block of rank 0
+            // (the heaviest, when causal), then rank 1, ...: the blocks running at
+            // any time share few K/V tensors (they stay in L2), and the light
+            // blocks of a group come last, where they fill the tail.
+            const int HB = p.H * p.B;
+            const int lin = (int)blockIdx.x + num_m * ((int)blockIdx.y + p.H * (int)blockIdx.z);
+            const int per_group = num_m * p.head_group;
+            const int gi = lin / per_group;
+            const int w = lin - gi * per_group;
+            const int hcnt = min(p.head_group, HB - gi * p.head_group);
+            blk = w / hcnt;
+            const int hb = gi * p.head_group + (w - blk * hcnt);
+            h = hb % p.H;
+            b = hb / p.H;
+        }
+    }
     const int m_blk = p.causal ? (num_m - 1 - blk) : blk;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
     const int m0 = m_blk * kBlockM;
     // this (b, h) problem's sizes, and where its rows start in the tensors
     int Nq_b = p.Nq, Nk_b = p.Nk, q_base = 0, k_base = 0;
