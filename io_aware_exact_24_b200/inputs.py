@@ -1,6 +1,7 @@
 """Seeded synthetic inputs for the attention forward (shared by tests, bench, oracle checks).
 
-This module only draws numbers and rounds them to bf16; it contains none of
+This module only draws numbers and rounds them to bf16 (or quantises them to
+8-bit E4M3 with a per-tensor scale); it contains none of
 the attention arithmetic, so both the CUDA path and the CPU oracle can consume
 its output without sharing any of the method's code.
 
@@ -144,6 +145,37 @@ def make_inputs(w: Workload):
     if w.key_len_range is not None:
         kl = key_lengths(w.B, w.key_len_range[0], w.key_len_range[1], w.seed)
     return {"q": q, "k": k, "v": v, "key_lens": kl}
+
+def normal_e4m3(shape, seed: int, tensor_id: int, sigma: float = 1.0):
+    """The same N(0, sigma^2) float32 samples as normal_bf16, stored as 8-bit E4M3
+    codes with one fp32 scale per tensor: scale = max|x| / 448 (448 is the largest
+    finite E4M3 value), codes = E4M3(x / scale) rounded to nearest even (torch's
+    float8_e4m3fn conversion).  Returns (uint8 codes, descale = scale as float)."""
+    import torch
+
+    x = _rng(seed, tensor_id).standard_normal(size=shape, dtype=np.float32)
+    if sigma != 1.0:
+        x *= np.float32(sigma)
+    amax = float(np.abs(x).max()) if x.size else 0.0
+    scale = np.float32(amax / 448.0) if amax > 0 else np.float32(1.0)
+    y = torch.from_numpy(np.ascontiguousarray(x / scale, dtype=np.float32))
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+    return codes, float(scale)
+
+
+def make_inputs_fp8(w: Workload):
+    """E4M3 inputs of workload w (the tensors make_inputs rounds to bf16, quantised
+    per tensor instead): dict(q8, k8, v8: uint8 [B,H,N,d]; q_descale, k_descale,
+    v_descale: float; key_lens: int32 [B] or None)."""
+    q8, qs = normal_e4m3((w.B, w.H, w.Nq, w.d), w.seed, TENSOR_Q, w.sigma)
+    k8, ks = normal_e4m3((w.B, w.H, w.Nk, w.d), w.seed, TENSOR_K, w.sigma)
+    v8, vs = normal_e4m3((w.B, w.H, w.Nk, w.d), w.seed, TENSOR_V, w.sigma)
+    kl = None
+    if w.key_len_range is not None:
+        kl = key_lengths(w.B, w.key_len_range[0], w.key_len_range[1], w.seed)
+    return {"q8": q8, "k8": k8, "v8": v8, "q_descale": qs, "k_descale": ks, "v_descale": vs,
+            "key_lens": kl}
+
 
 def alibi_slopes(H: int) -> np.ndarray:
     """The usual geometric per-head bias slopes 2^(-8(h+1)/H), fp32 [H]."""

@@ -200,3 +200,58 @@ def attn_online(q, k, v, scale, causal=False, key_lens=None, block=7):
     if rc != 0:
         raise RuntimeError(f"attn_online_fp64 failed ({rc})")
     return o, lse
+
+
+# --------------------------------------------------------------------------------------
+# FP8 (e4m3) inputs with per-tensor scales: "FlashAttention：把注意力从公式写成数据流",
+# section "精度、掩码和边界情况" (low-precision inputs; report the error against the
+# 16-bit result) and "FlashAttention 与边缘设备上的注意力内存瓶颈", section 3.3
+# (FP8 on the newest tensor cores).  What is computed is the attention of the
+# dequantised inputs: Q = q_descale * Q8, K = k_descale * K8, V = v_descale * V8.
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Decode 8-bit E4M3 codes (the OCP 8-bit floating point format, 'fn' flavour):
+    sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds
+    the subnormals m * 2^-9; no infinities; 0x7F and 0xFF are NaN (largest finite
+    value 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = sign * mag
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def e4m3_to_bf16_bits(codes) -> np.ndarray:
+    """The bf16 bit pattern of each E4M3 value (exact: 4 significant bits and
+    exponents -9..8 fit in bf16)."""
+    f = e4m3_to_f64(codes).astype(np.float32)
+    u = f.view(np.uint32)
+    finite = np.isfinite(f)
+    if np.any((u[finite] & np.uint32(0xFFFF)) != 0):
+        raise AssertionError("e4m3 value not exact in bf16")
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def _e4m3_scale(scale, q_descale, k_descale):
+    # Reading: the three fp32 factors of the scores are folded into one fp32 scale
+    # (a relative change of at most 2^-24 in every score).
+    return float(np.float32(np.float64(scale) * np.float64(q_descale) * np.float64(k_descale)))
+
+
+def attn_ref_e4m3(q8, k8, v8, scale, q_descale, k_descale, v_descale, causal=False, key_lens=None):
+    """Plain definition on dequantised e4m3 inputs (uint8 codes [B,H,N,d]):
+    softmax(scale * (qd Q8)(kd K8)^T) (vd V8) = vd * attn(Q8, K8, V8; scale*qd*kd).
+    Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq])."""
+    o, lse = attn_ref(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8), e4m3_to_bf16_bits(v8),
+                      _e4m3_scale(scale, q_descale, k_descale), causal, key_lens)
+    return o * np.float64(np.float32(v_descale)), lse
+
+
+def attn_ref_rows_e4m3(q8, k8, v8, scale, q_descale, k_descale, v_descale, row_ids, causal=False,
+                       key_lens=None):
+    """attn_ref_e4m3 on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n])."""
+    o, lse = attn_ref_rows(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8), e4m3_to_bf16_bits(v8),
+                           _e4m3_scale(scale, q_descale, k_descale), row_ids, causal, key_lens)
+    return o * np.float64(np.float32(v_descale)), lse

@@ -56,3 +56,20 @@ def test_window_flop_counts_visible_pairs():
         pairs = sum(1 for i in range(Nq) for j in range(Nk)
                     if j >= i + Nk - Nq - W and (not causal or j <= i + Nk - Nq))
         assert w.flop == 4.0 * 2 * 3 * 8 * pairs
+
+
+def test_e4m3_inputs_are_the_bf16_tensors_quantised():
+    import oracle
+    from io_aware_exact_24_b200.inputs import normal_e4m3
+
+    shape = (2, 3, 70, 64)
+    codes, s = normal_e4m3(shape, 4, 1, 0.5)
+    x = np.random.Generator(np.random.Philox(key=4 * 16 + 1)).standard_normal(size=shape, dtype=np.float32)
+    x = x * np.float32(0.5)
+    assert np.float32(s) == np.float32(np.abs(x).max() / 448.0)
+    y = oracle.e4m3_to_f64(codes) * s
+    # round to nearest: half an ulp, 2^-4 relative for normals, 2^-10 * s absolute below 2^-6 * s
+    err = np.abs(y - x.astype(np.float64))
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    assert np.abs(oracle.e4m3_to_f64(codes)).max() == 448.0   # the largest |x| maps to 448

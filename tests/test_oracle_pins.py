@@ -388,3 +388,92 @@ def test_varlen_of_equal_lengths_is_the_dense_problem():
     ov, lv = oracle.attn_ref_varlen(pack(q), pack(k), pack(v), cu, cu, 0.3, True)
     assert np.array_equal(ov, o.transpose(0, 2, 1, 3).reshape(B * N, H, d))
     assert np.array_equal(lv, lse.transpose(0, 2, 1).reshape(B * N, H))
+
+
+# ---------------------------------------------------------------- e4m3 inputs
+# Pins of the FP8 wrapper: the code decode against a library conversion and the
+# format's closed forms, and the algebra of the three descales against the
+# (already pinned) bf16 oracle on the same values.
+
+def test_e4m3_decode_matches_torch_on_all_codes():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(ours[fin], ref[fin])
+    assert np.array_equal(np.signbit(ours[fin]), np.signbit(ref[fin]))
+
+
+def test_e4m3_closed_forms():
+    d = oracle.e4m3_to_f64(np.array([0x00, 0x80, 0x38, 0xB8, 0x7E, 0xFE, 0x01, 0x07, 0x08, 0x7F, 0xFF],
+                                    np.uint8))
+    assert d[0] == 0 and not np.signbit(d[0]) and d[1] == 0 and np.signbit(d[1])
+    assert d[2] == 1.0 and d[3] == -1.0
+    assert d[4] == 448.0 and d[5] == -448.0          # largest finite: 1.75 * 2^8
+    assert d[6] == 2.0 ** -9 and d[7] == 7 * 2.0 ** -9  # subnormals m * 2^-9
+    assert d[8] == 2.0 ** -6                          # smallest normal
+    assert np.isnan(d[9]) and np.isnan(d[10])
+    bits = oracle.e4m3_to_bf16_bits(np.array([0x38, 0x7E, 0x01], np.uint8))
+    assert list(bits) == [0x3F80, 0x43E0, 0x3B00]
+
+
+def _codes(shape, seed):
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x38                      # no NaN codes
+    return c
+
+
+@pytest.mark.parametrize("causal,kl", [(False, None), (True, None), (False, [5, 40])])
+def test_e4m3_unit_descales_are_the_bf16_oracle(causal, kl):
+    B, H, Nq, Nk, d = 2, 2, 33, 40, 16
+    q8 = _codes((B, H, Nq, d), 1) & 0xBF              # exponents <= 7: moderate scores
+    k8 = _codes((B, H, Nk, d), 2) & 0xBF
+    v8 = _codes((B, H, Nk, d), 3)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.03125, 1.0, 1.0, 1.0, causal, kl_arr)
+    qf, kf, vf = (oracle.e4m3_to_f64(x).astype(np.float32) for x in (q8, k8, v8))
+    o2, l2 = oracle.attn_ref(_bits(qf), _bits(kf), _bits(vf), 0.03125, causal, kl_arr)
+    assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+
+
+def test_e4m3_descales_scale_scores_and_values():
+    B, H, Nq, Nk, d = 1, 2, 20, 24, 8
+    q8 = _codes((B, H, Nq, d), 4) & 0xBF
+    k8 = _codes((B, H, Nk, d), 5) & 0xBF
+    v8 = _codes((B, H, Nk, d), 6)
+    base_o, base_l = oracle.attn_ref_e4m3(q8, k8, v8, 0.02, 1.0, 1.0, 1.0)
+    # q and k descales multiply the scores: (2, 0.5) is (1, 1); (2, 1) is scale * 2
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.02, 2.0, 0.5, 1.0)
+    assert np.array_equal(o, base_o) and np.array_equal(lse, base_l)
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.02, 2.0, 1.0, 1.0)
+    o2, l2 = oracle.attn_ref_e4m3(q8, k8, v8, 0.04, 1.0, 1.0, 1.0)
+    assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+    assert not np.allclose(lse, base_l)
+    # the v descale multiplies O and leaves the LSE alone
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.02, 1.0, 1.0, 0.25)
+    assert np.array_equal(o, base_o * 0.25) and np.array_equal(lse, base_l)
+
+
+def test_e4m3_zero_query_gives_the_scaled_mean_of_values():
+    B, H, Nq, Nk, d = 1, 1, 6, 10, 8
+    q8 = np.zeros((B, H, Nq, d), np.uint8)
+    k8 = _codes((B, H, Nk, d), 7)
+    v8 = _codes((B, H, Nk, d), 8)
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.1, 3.0, 5.0, 0.5, causal=True)
+    vf = oracle.e4m3_to_f64(v8)[0, 0]
+    for i in range(Nq):
+        n = i + (Nk - Nq) + 1
+        np.testing.assert_allclose(o[0, 0, i], 0.5 * vf[:n].mean(axis=0), rtol=0, atol=1e-12)
+        assert abs(lse[0, 0, i] - math.log(n)) < 1e-13
+
+
+def test_e4m3_rows_entry_matches_full_evaluation():
+    B, H, Nq, Nk, d = 2, 2, 17, 23, 16
+    q8, k8, v8 = _codes((B, H, Nq, d), 9) & 0xBF, _codes((B, H, Nk, d), 10) & 0xBF, _codes((B, H, Nk, d), 11)
+    o, lse = oracle.attn_ref_e4m3(q8, k8, v8, 0.05, 1.5, 0.75, 2.0, True)
+    rows = np.array([0, 5, 16, 17, 40, 67], np.int64)
+    orow, lrow = oracle.attn_ref_rows_e4m3(q8, k8, v8, 0.05, 1.5, 0.75, 2.0, rows, True)
+    assert np.array_equal(orow, o.reshape(-1, d)[rows]) and np.array_equal(lrow, lse.reshape(-1)[rows])
