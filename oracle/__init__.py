@@ -204,9 +204,9 @@ def attn_online(q, k, v, scale, causal=False, key_lens=None, block=7):
 
 # --------------------------------------------------------------------------------------
 # FP8 (e4m3) inputs with per-tensor scales: "FlashAttention：把注意力从公式写成数据流",
-# section "精度、掩码和边界情况" (low-precision inputs; report the error against the
-# 16-bit result) and "FlashAttention 与边缘设备上的注意力内存瓶颈", section 3.3
-# (FP8 on the newest tensor cores).  What is computed is the attention of the
+# section "FA2 与 FA3" (the Hopper kernel brings low-precision arithmetic in) and
+# section "用实验验证而不是背诵结论" (FP8 saves HBM bytes but needs scaling; report
+# its error against a 16-bit baseline).  What is computed is the attention of the
 # dequantised inputs: Q = q_descale * Q8, K = k_descale * K8, V = v_descale * V8.
 
 def e4m3_to_f64(codes) -> np.ndarray:
