@@ -31,7 +31,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from io_aware_exact_24_b200.inputs import (DECODE_WORKLOADS, WINDOW_WORKLOADS,  # noqa: E402
-                                           WORKLOADS, WORKLOAD_ORDER, make_inputs)
+                                           WORKLOADS, WORKLOAD_ORDER, make_inputs,
+                                           make_inputs_fp8)
 
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -227,6 +228,57 @@ def window_table(steps, warmup, device, peak_tflops):
                                                 "frac": tf / peak_tflops},
                      "flop": ("4*B*H*d*(visible query-key pairs)" if w.window_left >= 0
                               else "4*B*H*Nq*Nk*d, causal halved"),
+                     "config": config_of(w, "flushed between timed launches", "single GPU")}
+        del x
+    return out
+
+
+def time_fp8(w, x, steps, warmup, device):
+    """Mean per-launch device time (ms) of fa_fwd_fp8 on resident E4M3 inputs, L2 flushed."""
+    import torch
+    from io_aware_exact_24_b200 import fa_fwd_fp8
+    q8, k8, v8 = (torch.from_numpy(np.ascontiguousarray(x[n])).to(device) for n in ("q8", "k8", "v8"))
+    kl = None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).to(device)
+    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        fa_fwd_fp8(q8, k8, v8, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, x["q_descale"],
+                   x["k_descale"], x["v_descale"], w.causal, kl, stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for st, en in ev:
+        flush.zero_()
+        st.record(stream)
+        launch()
+        en.record(stream)
+    torch.cuda.synchronize()
+    per = [st.elapsed_time(en) for st, en in ev]
+    del q8, k8, v8, o, lse, flush
+    return float(np.mean(per))
+
+
+def fp8_table(steps, warmup, device, peak_bf16_tflops):
+    """E4M3 inputs (fa_fwd_fp8) on the d = 128 workloads.  The roofline peak is the
+    measured bf16 peak times the nominal FP8 / BF16 dense ratio (4.5 / 2.25 = 2)."""
+    out = {}
+    for name in ("causal_8000_d128",):
+        w = WORKLOADS[name]
+        x = make_inputs_fp8(w)
+        ms = time_fp8(w, x, steps, warmup, device)
+        tf = w.flop / (ms / 1000.0) / 1e12
+        peak = 2.0 * peak_bf16_tflops
+        out[name] = {"entry": "fa_fwd_fp8", "dtype": "e4m3 in, bf16 out", "ms": ms, "tflops": tf,
+                     "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                  "frac": tf / peak,
+                                  "peak_basis": "measured bf16 x nominal fp8/bf16 ratio 2"},
                      "config": config_of(w, "flushed between timed launches", "single GPU")}
         del x
     return out
@@ -541,6 +593,7 @@ def main():
                                               float(peaks["hbm_gbs"]))
         line["sliding_window"] = window_table(args.steps, args.warmup, device, peak)
         line["varlen"] = varlen_table(args.steps, args.warmup, device, peak)
+        line["fp8"] = fp8_table(args.steps, args.warmup, device, peak)
         cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
         rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",

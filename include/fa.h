@@ -133,6 +133,34 @@ FA_API int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, flo
                 fa_stream_t stream);
 
 /*
+ * fa_fwd_fp8 -- fa_fwd on 8-bit E4M3 inputs with per-tensor scales: computes
+ * the attention of the dequantised tensors Q = q_descale * Q8,
+ * K = k_descale * K8, V = v_descale * V8, i.e.
+ *   O = softmax(scale * Q K^T + mask) V,  LSE as fa_fwd,
+ * with E4M3 tensor-core products (the low-precision arithmetic the Hopper
+ * kernel brings in, "FlashAttention：把注意力从公式写成数据流", section
+ * "FA2 与 FA3"; FP8 saves HBM bytes but needs scaling and an error report
+ * against a 16-bit baseline, same page, section "用实验验证而不是背诵结论").
+ * The probabilities are rounded to E4M3 before the PV product and O is
+ * normalised by the sum of those rounded values, so O's error is set by P's
+ * 3-bit mantissa; the LSE uses the unrounded sum.
+ *
+ *   q8, k8, v8  device uint8 E4M3 codes (OCP 8-bit float, no infinities,
+ *               0x7F/0xFF NaN), [B,H,N_q|N_k|N_k,d] contiguous, 16-byte aligned.
+ *   o           device bf16 [B,H,N_q,d], 16-byte aligned.
+ *   lse         device fp32 [B,H,N_q], 4-byte aligned.
+ *   d           128 only (FA_ERR_UNSUPPORTED otherwise).
+ *   q_descale, k_descale, v_descale   finite, > 0 (FA_ERR_INVALID_ARG
+ *               otherwise); scale * q_descale * k_descale is rounded once to
+ *               fp32 and must stay finite and > 0.
+ *   other arguments, ownership, empty cases and errors as fa_fwd.
+ */
+FA_API int fa_fwd_fp8(const void *q8, const void *k8, const void *v8, void *o, float *lse,
+               int B, int H, int N_q, int N_k, int d, float scale, float q_descale,
+               float k_descale, float v_descale, int causal, const int32_t *key_lens,
+               fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- attention over a batch of sequences of different lengths
  * packed back to back without padding (the packed variable-length batches of
  * the mask variants, "FlashAttention：把注意力从公式写成数据流", section

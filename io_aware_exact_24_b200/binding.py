@@ -61,6 +61,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                         vp, vp, i32, vp]
             lib.fa_fwd_bias.restype = i32
+            lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32,
+                                       f32, i32, vp, vp]
+            lib.fa_fwd_fp8.restype = i32
             lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                           f32, i32, vp]
             lib.fa_fwd_varlen.restype = i32
@@ -159,6 +162,18 @@ def fa_fwd_bias(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, slo
                                     int(window_left), _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_bias")
+    return st
+
+
+def fa_fwd_fp8(q8, k8, v8, o, lse, B, H, N_q, N_k, d, scale, q_descale, k_descale, v_descale,
+               causal, key_lens, stream=None, check=True) -> int:
+    """``fa_fwd_fp8`` of include/fa.h: forward on E4M3 inputs with per-tensor descales."""
+    st = load_library().fa_fwd_fp8(_addr(q8), _addr(k8), _addr(v8), _addr(o), _addr(lse),
+                                   int(B), int(H), int(N_q), int(N_k), int(d), float(scale),
+                                   float(q_descale), float(k_descale), float(v_descale),
+                                   int(bool(causal)), _addr(key_lens), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8")
     return st
 
 

@@ -95,6 +95,9 @@ int prepare_device(int dev) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128, true>::kSmemBytes);
         if (e != cudaSuccess) {
             st.status = cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
             return;
@@ -130,16 +133,19 @@ int validate(const void* q, const void* k, const void* v, const void* o, const v
     return FA_OK;
 }
 
-// [B,H,N,d] bf16 viewed as a 4-D tensor (d, N, H, B), box 64 x 128 x 1 x 1, 128B swizzle.
-bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d) {
+// [B,H,N,d] viewed as a 4-D tensor (d, N, H, B), 128B swizzle, box of one 128-byte
+// row segment x 128 rows: 64 bf16 columns, or (e4m3 = true) 128 one-byte columns.
+bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, bool e4m3 = false) {
     EncodeTiledFn enc = encoder();
     if (enc == nullptr) return false;
+    const cuuint64_t eb = e4m3 ? 1 : 2;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2, (cuuint64_t)H * N * d * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)fa::kBlockM, 1, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * eb, (cuuint64_t)N * d * eb, (cuuint64_t)H * N * d * eb};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), (cuuint32_t)fa::kBlockM, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -200,18 +206,19 @@ int launch_varlen(const void* q, const void* k, const void* v, void* o, float* l
     return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (packed variable-length)", e);
 }
 
-template <int D>
+// kF8: E4M3 Q, K, V (plain single-pass path only); o_scale multiplies O.
+template <int D, bool kF8 = false>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
            float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr},
-           int window_left = -1, const float* slopes = nullptr) {
+           int window_left = -1, const float* slopes = nullptr, float o_scale = 1.f) {
     CUtensorMap tq, tk, tv, to;
     // With no keys the K/V maps are never read; give them a valid 1-row shape.
     const void* kp = N_k > 0 ? k : q;
     const void* vp = N_k > 0 ? v : q;
     const int nk_map = N_k > 0 ? N_k : 1;
     const int b_kv = N_k > 0 ? B : 1, h_kv = N_k > 0 ? H : 1;
-    if (!encode_bhnd(&tq, q, B, H, N_q, D) || !encode_bhnd(&tk, kp, b_kv, h_kv, nk_map, D) ||
-        !encode_bhnd(&tv, vp, b_kv, h_kv, nk_map, D) || !encode_bhnd(&to, o, B, H, N_q, D)) {
+    if (!encode_bhnd(&tq, q, B, H, N_q, D, kF8) || !encode_bhnd(&tk, kp, b_kv, h_kv, nk_map, D, kF8) ||
+        !encode_bhnd(&tv, vp, b_kv, h_kv, nk_map, D, kF8) || !encode_bhnd(&to, o, B, H, N_q, D)) {
         snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
         return FA_ERR_CUDA;
     }
@@ -230,6 +237,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.num_splits = sp.num_splits > 0 ? sp.num_splits : 1;
     p.o_part = sp.o_part;
     p.lse_part = sp.lse_part;
+    p.o_scale = o_scale;
     const int rows_per_cta = fa::kBlockM;
     const unsigned num_m = (unsigned)((N_q + rows_per_cta - 1) / rows_per_cta);
     if (sp.num_splits <= 0 && causal && num_m >= kHeadGroupMinBlocks) {
@@ -240,6 +248,13 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         const long long hb = (long long)H * B;
         p.head_group = (int)(hg < 1 ? 1 : (hg > hb ? hb : hg));
     }
+    if constexpr (kF8) {
+        dim3 grid(num_m, (unsigned)H, (unsigned)B);
+        fa::fa_fwd_sm100_kernel<D, false, false, true>
+            <<<grid, fa::kNumThreads, fa::Cfg<D, true>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        const cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (e4m3)", e);
+    } else {
     if (sp.num_splits <= 0) {
         dim3 grid(num_m, (unsigned)H, (unsigned)B);
         fa::fa_fwd_sm100_kernel<D, false><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
@@ -255,6 +270,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         sp.o_part, sp.lse_part, reinterpret_cast<__nv_bfloat16*>(o), lse, rows, sp.num_splits);
     e = cudaGetLastError();
     return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV combine)", e);
+    }
 }
 
 constexpr int kMaxSplits = 256;
@@ -480,6 +496,35 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
     const SplitParts none{0, nullptr, nullptr};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H, int N_q, int N_k,
+               int d, float scale, float q_descale, float k_descale, float v_descale, int causal,
+               const int32_t* key_lens, fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q8, k8, v8, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    for (const float x : {q_descale, k_descale, v_descale})
+        if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
+    // the scores' three factors, folded into the one scale the kernel applies
+    const float c = scale * q_descale * k_descale;
+    if (!(c * 1.4426950408889634f > 0.f) || !std::isfinite(c * 1.4426950408889634f)) return FA_ERR_INVALID_ARG;
+    if (empty) return FA_OK;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const SplitParts none{0, nullptr, nullptr};
+    return launch<128, true>(q8, k8, v8, o, lse, B, H, N_q, N_k, c, causal, key_lens, s, none, -1, nullptr,
+                             v_descale);
 }
 
 int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,

@@ -104,27 +104,38 @@ struct FwdParams {
     // dense single-pass mode: > 1 reorders the CTAs' work (see the kernel); 0 or 1 keeps
     // blockIdx = (query block, h, b)
     int head_group;
+    // E4M3 mode only: the V descale, applied to O in the epilogue
+    float o_scale;
 };
 
-template <int D>
+// kF8 = false: bf16 Q, K, V and P (kind::f16 MMAs).  kF8 = true: E4M3 Q, K, V
+// with per-tensor descales, P rounded to E4M3 (kind::f8f6f4 MMAs, K = 32 per
+// instruction); d = 128 only, so a row is one 128-byte swizzle row.
+template <int D, bool kF8 = false>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static constexpr int kBoxes = D / 64;                        // 64-column boxes per row
-    static constexpr int kTileBytes = kBlockM * D * 2;           // one Q / K / V tile
-    static constexpr int kStagesK = (D == 64) ? 4 : 2;           // K ring slots
-    static constexpr int kStagesV = (D == 64) ? 4 : 2;           // V ring slots
-    // A V slot holds the tile (kBoxes 64-column boxes) followed by one box of
-    // bf16 ones: the PV product runs with N = D + 16 and its last 16 output
-    // columns accumulate the row sums of the bf16 P it multiplies.
+    static_assert(!kF8 || D == 128, "E4M3 inputs: d = 128");
+    static constexpr int kElemBytes = kF8 ? 1 : 2;
+    static constexpr int kBoxCols = 128 / kElemBytes;            // elements per 128-byte box row
+    static constexpr int kBoxes = D * kElemBytes / 128;          // boxes per Q / K / V row
+    static constexpr int kOBoxes = D / 64;                       // boxes per bf16 O row
+    static constexpr int kTileBytes = kBlockM * D * kElemBytes;  // one Q / K / V tile
+    static constexpr int kKPerMma = 32 / kElemBytes;             // K extent of one MMA (32 bytes)
+    static constexpr int kStagesK = (kTileBytes == 16384) ? 4 : 2;   // K ring slots
+    static constexpr int kStagesV = (kTileBytes == 16384) ? 4 : 2;   // V ring slots
+    // A V slot holds the tile (kBoxes boxes) followed by one box of ones: the
+    // PV product runs with N = D + 16 and its last 16 output columns
+    // accumulate the row sums of the rounded P it multiplies.
     static constexpr int kVSlotBytes = kTileBytes + kSwizzleBoxBytes;
+    static constexpr uint32_t kOnesWord = kF8 ? 0x38383838u : 0x3F803F80u;   // 1.0 in E4M3 / bf16
     static constexpr int kNPV = D + 16;
     static constexpr int kStages = kStagesK + kStagesV;
     // Of every 8 pairs of probabilities, this many are computed on the FMA pipe
     // (exp2_fma2) and the rest on MUFU, so neither unit is the lone bottleneck.
 #ifdef FA_EMU_PAIRS_D64
-    static constexpr int kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
+    static constexpr int kEmuPairs = (D == 64 || kF8) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
 #else
-    static constexpr int kEmuPairs = (D == 64) ? 2 : 0;   // measured best on B200
+    static constexpr int kEmuPairs = (D == 64 || kF8) ? 2 : 0;   // measured best on B200
 #endif
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kTileBytes;
@@ -142,22 +153,27 @@ struct Cfg {
     static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, lu [2][row] each
     static constexpr int kSmemBytes = kEpiOff + 2 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
-    // TMEM columns: the S buffer at 0..127, the P buffers (bf16 pairs, 64
-    // each) at 128..319, O at 320..320+D-1 and its row-sum columns right
-    // after (320+D .. 320+D+15); the O rescale also touches the 16 unused
-    // columns after those (at most column 479).
+    // The bf16 O tile is staged for its TMA store from the start of the Q
+    // buffer on; with 8-bit inputs it also covers the first K slot (idle by then).
+    static_assert(kOBoxes * kSwizzleBoxBytes <= kVOff, "O staging area");
+    // TMEM columns: the S buffer at 0..127, the P buffers (kPCols each: bf16
+    // pairs or E4M3 quads) after it, then O (D columns) and its row-sum
+    // columns; the O rescale also touches the 16 unused columns after those.
+    static constexpr uint32_t kPCols = kBlockN * kElemBytes / 4;
     __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
-    __host__ __device__ static constexpr uint32_t col_p(int b) { return 128u * kSBufs + 64u * b; }
-    static constexpr uint32_t kColO = 128u * kSBufs + 64u * kPBufs;
-    static constexpr uint32_t kColL = kColO + D;                 // row sum of the bf16 P
+    __host__ __device__ static constexpr uint32_t col_p(int b) { return 128u * kSBufs + kPCols * b; }
+    static constexpr uint32_t kColO = 128u * kSBufs + kPCols * kPBufs;
+    static constexpr uint32_t kColL = kColO + D;                 // row sum of the rounded P
     static_assert(kColO + D + 32 <= 512, "TMEM columns");
-    // Instruction descriptors (kind::f16): D=f32, A=B=bf16, M=128.
+    // Instruction descriptors: D = f32, M = 128; A/B format 1 = bf16 (kind::f16)
+    // or 0 = E4M3 (kind::f8f6f4).
     //   QK^T: A=Q K-major, B=K K-major, N=128.
     //   PV: A=P (TMEM, K-major), B=[V | ones] MN-major, N=D+16.
-    static constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
+    static constexpr uint32_t kFmt = kF8 ? 0u : 1u;
+    static constexpr uint32_t kIdescQK = (1u << 4) | (kFmt << 7) | (kFmt << 10) | (0u << 15) |
                                          (0u << 16) | ((uint32_t)(kBlockN >> 3) << 17) |
                                          ((uint32_t)(kBlockM >> 4) << 24);
-    static constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) |
+    static constexpr uint32_t kIdescPV = (1u << 4) | (kFmt << 7) | (kFmt << 10) | (0u << 15) |
                                          (1u << 16) | ((uint32_t)(kNPV >> 3) << 17) |
                                          ((uint32_t)(kBlockM >> 4) << 24);
 };
@@ -213,18 +229,21 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
     return e;
 }
 
-// p = 2^(s*c - mu) for keys 64*h2 .. 64*h2+63 of the thread's row, packed to
-// bf16 pairs and stored to its TMEM lane at taddr_p + 32*h2.  lu sums the
-// unrounded p (for the log-sum-exp; the sum of the bf16-rounded p, which
+// p = 2^(s*c - mu) for keys 64*h2 .. 64*h2+63 of the thread's row, rounded
+// to bf16 pairs (kF8 = false) or E4M3 quads (kF8 = true) and stored to its
+// TMEM lane: 32 (or 16) columns from taddr_p + 32*h2 (or 16*h2).  lu sums the
+// unrounded p (for the log-sum-exp; the sum of the rounded p, which
 // normalises O, comes out of the PV product).  kEmu of every 8 pairs go
 // through exp2_fma2, the rest through MUFU ex2 (which maps -inf to 0, so masked
-// tiles use kEmu = 0).
-template <int kEmu, int h2>
+// tiles use kEmu = 0).  p <= 2^8 (the reference-max threshold), inside E4M3's
+// range.
+template <int kEmu, int h2, bool kF8 = false>
 __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float c, float mu, uint32_t taddr_p,
                                                float2& lu) {
     const float2 c2 = make_float2(c, c);
     const float2 nmu = make_float2(-mu, -mu);
-    uint32_t w[32];
+    uint32_t w[kF8 ? 16 : 32];
+    float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int pi = 32 * h2 + i;
@@ -236,11 +255,20 @@ __device__ __forceinline__ void exp_store_half(const float (&s)[kBlockN], float 
             e.x = ex2_approx(x.x);
             e.y = ex2_approx(x.y);
         }
-        w[i] = pack_bf16x2(e.x, e.y);
+        if constexpr (kF8) {
+            if (i & 1)
+                w[i >> 1] = pack_e4m3x4(prev.x, prev.y, e.x, e.y);
+            else
+                prev = e;
+        } else {
+            w[i] = pack_bf16x2(e.x, e.y);
+        }
         lu = __fadd2_rn(lu, e);
     }
-
-    tmem_st32(taddr_p + 32u * h2, w);
+    if constexpr (kF8)
+        tmem_st16(taddr_p + 16u * h2, w);
+    else
+        tmem_st32(taddr_p + 32u * h2, w);
 }
 
 // Maximum of s[o .. o+31] as a tree of three-input max (depth 4).
@@ -276,12 +304,15 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
 // fa_splitkv_combine_kernel.
 // kVarlen = true: packed variable-length batches (FwdParams::cu_q / cu_k);
 // the TMA maps then view [tokens, H, D] as (D, H, tokens, 1).
-template <int D, bool kSplit = false, bool kVarlen = false>
+// kF8 = true: E4M3 inputs (see Cfg); O is still bf16 and FwdParams::o_scale
+// (the V descale) multiplies it in the epilogue.
+template <int D, bool kSplit = false, bool kVarlen = false, bool kF8 = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                         const FwdParams p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, kF8>;
+    static_assert(!kF8 || (!kSplit && !kVarlen), "E4M3 inputs: dense single-pass mode");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -414,7 +445,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     for (int i = threadIdx.x; i < C::kStagesV * (kSwizzleBoxBytes / 16); i += kNumThreads) {
         const int sl = i / (kSwizzleBoxBytes / 16);
         const uint32_t a = ring_slot(1, sl) + (uint32_t)C::kTileBytes + (uint32_t)(i % (kSwizzleBoxBytes / 16)) * 16u;
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0x3F803F80u) : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(C::kOnesWord) : "memory");
     }
     fence_proxy_async_smem();   // visible to the tensor core's reads
     __syncthreads();
@@ -437,7 +468,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 int qc1, qc2, qc3;
                 tile_coords(q_base, m0, qc1, qc2, qc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * 64, qc1, qc2, qc3,
+                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * C::kBoxCols, qc1, qc2, qc3,
                                 policy_evict_first());
             }
             bool ok = true;
@@ -451,7 +482,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 int kc1, kc2, kc3;
                 tile_coords(k_base, (t0 + j) * kBlockN, kc1, kc2, kc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * 64, kc1, kc2,
+                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * C::kBoxCols, kc1, kc2,
                                 kc3, pol_kv);
             }
             if (!ok) {
@@ -481,11 +512,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     tc_fence_after();
                     const uint32_t slot = ring_slot(0, sl);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < D * C::kElemBytes / 32; ++kk) {
+                        // 32 bytes of every row per MMA: 4 steps per 128-byte box
                         const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
                         const uint64_t a = smem_desc_sw128(q_tile + koff, 16, 1024);
                         const uint64_t bb = smem_desc_sw128(slot + koff, 16, 1024);
-                        umma_ss(tmem + C::col_s(i % C::kSBufs), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
+                        if constexpr (kF8)
+                            umma_ss_f8(tmem + C::col_s(i % C::kSBufs), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
+                        else
+                            umma_ss(tmem + C::col_s(i % C::kSBufs), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(bar_s_full(i & 1));   // per softmax warp: tiles i, i+2, ...
                     umma_commit(bar_empty(0, sl));
@@ -502,12 +537,16 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     tc_fence_after();
                     const uint32_t slot = ring_slot(1, sl);
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                        // keys 16kk..16kk+15 of P: 8 bf16-pair columns per step
+                    for (int kk = 0; kk < kBlockN / C::kKPerMma; ++kk) {
+                        // keys kK*kk .. kK*kk+kK-1 of P (kK = 16 bf16 or 32 E4M3): 8 TMEM
+                        // columns of P, kK 128-byte rows of the V slot per step
                         const uint32_t a_col = C::col_p(pb) + (uint32_t)(kk * 8);
                         const uint64_t bb =
-                            smem_desc_sw128(slot + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024);
-                        umma_ts(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                            smem_desc_sw128(slot + (uint32_t)(kk * C::kKPerMma * 128), kSwizzleBoxBytes, 1024);
+                        if constexpr (kF8)
+                            umma_ts_f8(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                        else
+                            umma_ts(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(bar_pv_done(pb));
                     umma_commit(bar_empty(1, sl));
@@ -619,11 +658,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             float2 lu2 = make_float2(0.f, 0.f);
             const uint32_t taddr_p = tmem + lane_off + C::col_p(pb);
             if (masked) {
-                exp_store_half<0, 0>(s, cs, mu, taddr_p, lu2);
-                exp_store_half<0, 1>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<0, 0, kF8>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<0, 1, kF8>(s, cs, mu, taddr_p, lu2);
             } else {
-                exp_store_half<C::kEmuPairs, 0>(s, cs, mu, taddr_p, lu2);
-                exp_store_half<C::kEmuPairs, 1>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<C::kEmuPairs, 0, kF8>(s, cs, mu, taddr_p, lu2);
+                exp_store_half<C::kEmuPairs, 1, kF8>(s, cs, mu, taddr_p, lu2);
             }
             lu += lu2.x + lu2.y;
             // O holds tiles < j relative to m_prev.  Only when some row of this
@@ -696,7 +735,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 reg_after_wait(u[0]);
                 l_row = __uint_as_float(u[0]);
             }
-            const float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
+            float inv_l = (l_row > 0.f) ? 1.f / l_row : 0.f;
+            if constexpr (kF8) inv_l *= p.o_scale;
 #pragma unroll
             for (int q4 = 0; q4 < D / 64; ++q4) {
                 const int col0 = g * (D / 2) + 32 * q4;   // first O column of this chunk
@@ -771,7 +811,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         fence_proxy_async_smem();
         const bool any_bad = named_bar_or(kBarSoftmaxAll, kSoftmaxWarps * 32, !good);
         if (!kSplit && !kVarlen && !any_bad && threadIdx.x == 0) {
-            for (int bx = 0; bx < C::kBoxes; ++bx)
+            for (int bx = 0; bx < C::kOBoxes; ++bx)
                 tma_store_4d(&tm_o, q_tile + bx * kSwizzleBoxBytes, bx * 64, m0, h, b);
             bulk_commit_group();
             bulk_wait_group_read0();

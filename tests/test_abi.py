@@ -276,3 +276,41 @@ def test_varlen_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert varlen_call() == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- E4M3 entry point
+
+def fp8_call(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, Nq=8, Nk=8, d=128, scale=0.088, qd=0.01,
+             kd=0.02, vd=0.005, causal=1, key_lens=None)
+    a.update(kw)
+    return binding.fa_fwd_fp8(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"],
+                              a["Nk"], a["d"], a["scale"], a["qd"], a["kd"], a["vd"], a["causal"],
+                              a["key_lens"], stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=64), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(qd=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(kd=-1.0), binding.FA_ERR_INVALID_ARG),
+    (dict(vd=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(vd=float("inf")), binding.FA_ERR_INVALID_ARG),
+    (dict(qd=1e-30, kd=1e-30), binding.FA_ERR_INVALID_ARG),   # scale * qd * kd is 0 in fp32
+    (dict(qd=1e30, kd=1e30), binding.FA_ERR_INVALID_ARG),     # ... or inf
+    (dict(scale=-1.0), binding.FA_ERR_INVALID_ARG),
+    (dict(q=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(v=P + 4), binding.FA_ERR_MISALIGNED),
+    (dict(o=None), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0), binding.FA_OK),
+    (dict(Nq=0, d=64), binding.FA_ERR_UNSUPPORTED),
+])
+def test_fp8_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert fp8_call(**kw) == code
+
+
+def test_fp8_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert fp8_call() == binding.FA_ERR_NO_DEVICE
