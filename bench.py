@@ -509,6 +509,8 @@ def main():
                     help="skip the per-workload table, e2e and CPU baseline (profiling runs)")
     ap.add_argument("--decode", default=None, choices=sorted(DECODE_WORKLOADS),
                     help="time only the split-KV forward on this decode workload (profiling runs)")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="time only the E4M3 forward on causal_8000_d128 (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -541,6 +543,11 @@ def main():
                                        "frac": gbs / float(peaks["hbm_gbs"])},
                           "config": config_of(w, "flushed between timed launches", "single GPU")}),
               flush=True)
+        return 0
+    if args.fp8_only:
+        peaks, _ = load_peaks()
+        print(json.dumps({"fp8": fp8_table(args.steps, args.warmup, device,
+                                           float(peaks["bf16_tflops"]))}), flush=True)
         return 0
     w = WORKLOADS[args.workload]
     x = make_inputs(w)
