@@ -255,3 +255,7 @@ def attn_ref_rows_e4m3(q8, k8, v8, scale, q_descale, k_descale, v_descale, row_i
     o, lse = attn_ref_rows(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8), e4m3_to_bf16_bits(v8),
                            _e4m3_scale(scale, q_descale, k_descale), row_ids, causal, key_lens)
     return o * np.float64(np.float32(v_descale)), lse
+
+
+# Backward pass (gradients of the plain definition): numpy, in its own module.
+from .attn_bwd import attn_bwd_ref  # noqa: E402,F401

@@ -477,3 +477,88 @@ def test_e4m3_rows_entry_matches_full_evaluation():
     rows = np.array([0, 5, 16, 17, 40, 67], np.int64)
     orow, lrow = oracle.attn_ref_rows_e4m3(q8, k8, v8, 0.05, 1.5, 0.75, 2.0, rows, True)
     assert np.array_equal(orow, o.reshape(-1, d)[rows]) and np.array_equal(lrow, lse.reshape(-1)[rows])
+
+
+# ---------------------------------------------------------------- backward oracle
+# Pins of oracle.attn_bwd_ref: a library routine the case reduces to (torch float64
+# autograd through its scaled_dot_product_attention with a boolean mask), the
+# forward it recomputes equals the pinned forward, and properties fixed by the
+# mathematics (softmax-gradient rows sum to zero, key-shift invariance, a closed form).
+
+BWD_CASES = [
+    # B, H, Nq, Nk, d, causal, key_lens
+    (2, 2, 19, 23, 8, False, None),
+    (1, 3, 23, 23, 16, True, None),
+    (2, 2, 15, 30, 8, True, None),           # N_q < N_k: bottom-right diagonal
+    (2, 1, 17, 21, 8, False, [9, 21]),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=[str(c) for c in BWD_CASES])
+def test_bwd_matches_torch_autograd_float64(case):
+    torch = pytest.importorskip("torch")
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 61)
+    do = normal_bf16((B, H, Nq, d), 61, 5)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    scale = 0.37
+    dq, dk, dv = oracle.attn_bwd_ref(q, k, v, do, scale, causal, kl_arr)
+    tq, tk, tv = (torch.from_numpy(bf16_bits_to_f32(x).astype(np.float64)).requires_grad_(True)
+                  for x in (q, k, v))
+    tdo = torch.from_numpy(bf16_bits_to_f32(do).astype(np.float64))
+    mask = np.stack([_visible(Nq, Nk, causal, Nk if kl is None else kl[b]) for b in range(B)])
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=torch.from_numpy(mask)[:, None], scale=float(np.float32(scale)))
+    out.backward(tdo)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_bwd_recomputed_forward_is_the_pinned_forward():
+    q, k, v = _rand(2, 2, 21, 26, 16, 62)
+    do = normal_bf16((2, 2, 21, 16), 62, 5)
+    kl = np.array([0, 20], np.int32)
+    _, _, _, parts = oracle.attn_bwd_ref(q, k, v, do, 0.25, True, kl, return_parts=True)
+    o, _ = oracle.attn_ref(q, k, v, 0.25, True, kl)
+    np.testing.assert_allclose(np.stack(parts["O"]).reshape(o.shape), o, rtol=0, atol=1e-13)
+
+
+def test_bwd_key_gradients_sum_to_zero_and_masked_keys_get_none():
+    B, H, Nq, Nk, d = 2, 2, 20, 28, 8
+    q, k, v = _rand(B, H, Nq, Nk, d, 63)
+    do = normal_bf16((B, H, Nq, d), 63, 5)
+    kl = np.array([28, 11], np.int32)
+    dq, dk, dv = oracle.attn_bwd_ref(q, k, v, do, 0.3, True, kl)
+    # each row of dS sums to zero, so sum_j dK_j = scale * sum_i (sum_j dS_ij) Q_i = 0
+    assert np.abs(dk.sum(axis=2)).max() < 1e-12
+    # keys past key_len are never visible: no gradient reaches them
+    assert np.all(dk[1, :, 11:] == 0) and np.all(dv[1, :, 11:] == 0)
+
+
+def test_bwd_key_shift_leaves_every_gradient_unchanged():
+    B, H, Nq, Nk, d = 1, 2, 12, 16, 8
+    rng = np.random.default_rng(64)
+    q = _bits(rng.integers(-3, 4, (B, H, Nq, d)).astype(np.float32) / 4)
+    k = _bits(rng.integers(-3, 4, (B, H, Nk, d)).astype(np.float32) / 4)
+    v = _bits(rng.integers(-3, 4, (B, H, Nk, d)).astype(np.float32) / 4)
+    do = _bits(rng.integers(-3, 4, (B, H, Nq, d)).astype(np.float32) / 4)
+    w = rng.integers(-2, 3, d).astype(np.float32) / 2
+    k2 = _bits(bf16_bits_to_f32(k) + w)
+    g1 = oracle.attn_bwd_ref(q, k, v, do, 0.5, True)
+    g2 = oracle.attn_bwd_ref(q, k2, v, do, 0.5, True)
+    for a, b in zip(g1, g2):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_bwd_zero_query_closed_form_for_dv():
+    B, H, Nq, Nk, d = 1, 2, 10, 10, 8
+    _, k, v = _rand(B, H, Nq, Nk, d, 65)
+    q = np.zeros((B, H, Nq, d), np.uint16)
+    do = normal_bf16((B, H, Nq, d), 65, 5)
+    _, _, dv = oracle.attn_bwd_ref(q, k, v, do, 0.9, True)
+    dof = bf16_bits_to_f32(do).astype(np.float64)
+    # P is uniform over keys 0..i: dV_j = sum_{i >= j} dO_i / (i + 1)
+    for j in range(Nk):
+        ref = sum(dof[0, :, i] / (i + 1) for i in range(j, Nq))
+        np.testing.assert_allclose(dv[0, :, j], ref, rtol=0, atol=1e-13)
