@@ -161,6 +161,44 @@ FA_API int fa_fwd_fp8(const void *q8, const void *k8, const void *v8, void *o, f
                fa_stream_t stream);
 
 /*
+ * fa_bwd -- backward pass of fa_fwd: given the upstream gradient dO of O, the
+ * gradients of O = softmax(scale * Q K^T + mask) V with respect to Q, K and V.
+ * The attention matrix is recomputed tile by tile from Q, K and the forward's
+ * LSE and never stored (the backward and its recomputation are named by
+ * "FlashAttention：把注意力从公式写成数据流", section "用实验验证而不是背诵结论",
+ * and "[2205.14135] FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness", section "三、FLOPs（計算能力）並非 Speedup 的主因素"):
+ *   P = exp(scale * Q K^T - LSE) on visible pairs, 0 elsewhere;
+ *   dV = P^T dO;  dS = P * (dO V^T - D), D_i = dO_i . O_i;
+ *   dQ = scale * dS K;  dK = scale * dS^T Q.
+ *
+ *   q, k, v       device bf16 [B,H,N_q|N_k|N_k,d], as given to fa_fwd.
+ *   o, lse        device: the outputs fa_fwd returned for these inputs (bf16
+ *                 [B,H,N_q,d], fp32 [B,H,N_q]).
+ *   dout          device bf16 [B,H,N_q,d], 16-byte aligned: dL/dO.
+ *   dq            device bf16 [B,H,N_q,d]; dk, dv device bf16 [B,H,N_k,d];
+ *                 16-byte aligned, written in full (rows of keys no query sees,
+ *                 and rows of queries that see no key, get 0).
+ *   B,H,N_q,N_k,d,scale,causal,key_lens   as for fa_fwd (same mask).
+ *   workspace     device, 256-byte aligned, at least fa_bwd_workspace_size(B,H,N_q,d)
+ *                 bytes, owned by the caller; overwritten (D and an fp32 dQ
+ *                 accumulator). Calls sharing a workspace must be ordered.
+ *   stream        as for fa_fwd; four launches are enqueued (D and zeroing, the
+ *                 main kernel, dQ to bf16).
+ *
+ * Returns FA_OK once enqueued.  Errors as fa_fwd, plus FA_ERR_INVALID_ARG for a
+ * NULL or short workspace or NULL gradient buffers, FA_ERR_MISALIGNED for
+ * unaligned dout/dq/dk/dv/workspace.  B = 0 or H = 0: no-op.  N_q = 0: dk = dv = 0.
+ * N_k = 0: dq = 0.  The dQ sums use atomic adds, so dq may differ in the last
+ * bits between runs; dk and dv are deterministic.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N_q, int d);
+FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dout, void *dq, void *dk, void *dv, int B, int H, int N_q, int N_k,
+           int d, float scale, int causal, const int32_t *key_lens, void *workspace,
+           size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- attention over a batch of sequences of different lengths
  * packed back to back without padding (the packed variable-length batches of
  * the mask variants, "FlashAttention：把注意力从公式写成数据流", section

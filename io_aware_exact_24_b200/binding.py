@@ -64,6 +64,11 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32,
                                        f32, i32, vp, vp]
             lib.fa_fwd_fp8.restype = i32
+            lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                   i32, vp, vp, sz, vp]
+            lib.fa_bwd.restype = i32
+            lib.fa_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
+            lib.fa_bwd_workspace_size.restype = sz
             lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                           f32, i32, vp]
             lib.fa_fwd_varlen.restype = i32
@@ -174,6 +179,22 @@ def fa_fwd_fp8(q8, k8, v8, o, lse, B, H, N_q, N_k, d, scale, q_descale, k_descal
                                    int(bool(causal)), _addr(key_lens), _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_fp8")
+    return st
+
+
+def fa_bwd_workspace_size(B, H, N_q, d) -> int:
+    return int(load_library().fa_bwd_workspace_size(int(B), int(H), int(N_q), int(d)))
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, d, scale, causal, key_lens,
+           workspace, workspace_bytes, stream=None, check=True) -> int:
+    """``fa_bwd`` of include/fa.h: gradients of the forward given dO (device workspace given)."""
+    st = load_library().fa_bwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(dout),
+                               _addr(dq), _addr(dk), _addr(dv), int(B), int(H), int(N_q), int(N_k),
+                               int(d), float(scale), int(bool(causal)), _addr(key_lens),
+                               _addr(workspace), int(workspace_bytes), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_bwd")
     return st
 
 

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace {
@@ -98,6 +99,12 @@ int prepare_device(int dev) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128, true>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::BwdCfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_bwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::BwdCfg<128>::kSmemBytes);
         if (e != cudaSuccess) {
             st.status = cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
             return;
@@ -314,6 +321,80 @@ HostLayout host_layout(int B, int H, int N_q, int N_k, int d, int has_key_lens) 
     return L;
 }
 
+// Workspace of the backward pass: D = rowsum(dO * O) [B,H,N_q] fp32, then the
+// fp32 dQ accumulator [B,H,N_q,d], each 256-byte aligned.
+struct BwdLayout {
+    size_t dsum, dq_acc, total;
+};
+BwdLayout bwd_layout(int B, int H, int N_q, int d) {
+    const size_t rows = (size_t)B * H * N_q;
+    BwdLayout L{};
+    L.dsum = 0;
+    L.dq_acc = round_up(rows * 4, 256);
+    L.total = L.dq_acc + round_up(rows * d * 4, 256);
+    return L;
+}
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, int B, int H, int N_q, int N_k, float scale, int causal,
+               const int32_t* key_lens, uint8_t* ws, cudaStream_t stream) {
+    const BwdLayout L = bwd_layout(B, H, N_q, D);
+    float* dsum = reinterpret_cast<float*>(ws + L.dsum);
+    float* dq_acc = reinterpret_cast<float*>(ws + L.dq_acc);
+    const long long rows = (long long)B * H * N_q;
+    cudaError_t e;
+    if (rows > 0) {
+        fa::fa_bwd_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+            reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), dsum, dq_acc,
+            rows);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("kernel launch (backward preprocessing)", e);
+    }
+    const size_t kv_bytes = (size_t)B * H * N_k * D * 2;
+    if (N_k > 0 && N_q == 0) {
+        // no query: no gradient reaches K or V
+        e = cudaMemsetAsync(dk, 0, kv_bytes, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, stream);
+        if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync", e);
+    }
+    if (N_k > 0 && N_q > 0) {
+        CUtensorMap tq, tk, tv, tdo;
+        if (!encode_bhnd(&tq, q, B, H, N_q, D) || !encode_bhnd(&tk, k, B, H, N_k, D) ||
+            !encode_bhnd(&tv, v, B, H, N_k, D) || !encode_bhnd(&tdo, dout, B, H, N_q, D)) {
+            snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
+            return FA_ERR_CUDA;
+        }
+        fa::BwdParams p{};
+        p.lse = lse;
+        p.dsum = dsum;
+        p.dq_acc = dq_acc;
+        p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+        p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+        p.key_lens = key_lens;
+        p.B = B;
+        p.H = H;
+        p.Nq = N_q;
+        p.Nk = N_k;
+        p.scale = scale;
+        p.scale_log2 = scale * 1.4426950408889634f;
+        p.causal = causal ? 1 : 0;
+        p.wait_limit = kWaitLimitCycles;
+        dim3 grid((unsigned)((N_k + 127) / 128), (unsigned)H, (unsigned)B);
+        fa::fa_bwd_sm100_kernel<D><<<grid, fa::kBwdThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("kernel launch (backward)", e);
+    }
+    if (rows > 0) {
+        const long long n8 = rows * D / 8;
+        fa::fa_bwd_post_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
+            dq_acc, reinterpret_cast<__nv_bfloat16*>(dq), scale, n8);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("kernel launch (backward dQ)", e);
+    }
+    return FA_OK;
+}
+
 __global__ void selftest_wait_kernel(unsigned long long limit) {
     __shared__ __align__(8) uint64_t bar;
     __shared__ int abort_flag;
@@ -525,6 +606,45 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* l
     const SplitParts none{0, nullptr, nullptr};
     return launch<128, true>(q8, k8, v8, o, lse, B, H, N_q, N_k, c, causal, key_lens, s, none, -1, nullptr,
                              v_descale);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N_q, int d) {
+    if (B < 0 || H < 0 || N_q < 0 || (d != 64 && d != 128)) return 0;
+    return bwd_layout(B, H, N_q, d).total;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int H, int N_q, int N_k, int d, float scale, int causal,
+           const int32_t* key_lens, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (B == 0 || H == 0) return FA_OK;
+    // with N_q = 0 only dK = dV = 0 are written; validate() stopped before the pointers
+    if (N_k > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)) return FA_ERR_INVALID_ARG;
+    if (N_q > 0 && (q == nullptr || o == nullptr || lse == nullptr || dout == nullptr || dq == nullptr))
+        return FA_ERR_INVALID_ARG;
+    if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16)) return FA_ERR_MISALIGNED;
+    if (N_k > 0 && (!aligned(k, 16) || !aligned(v, 16))) return FA_ERR_MISALIGNED;
+    if (key_lens != nullptr && !aligned(key_lens, 4)) return FA_ERR_MISALIGNED;
+    const BwdLayout L = bwd_layout(B, H, N_q, d);
+    if (workspace == nullptr || workspace_bytes < L.total) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (d == 64)
+        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s);
 }
 
 int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,

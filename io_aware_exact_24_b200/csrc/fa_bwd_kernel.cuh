@@ -1,0 +1,460 @@
+// fa_bwd_kernel.cuh -- attention backward pass for sm_100a (B200).
+//
+// What it computes: given Q, K, V, the forward's O and LSE, and the upstream
+// gradient dO, the gradients of O = softmax(scale * Q K^T + mask) V:
+//   P  = exp(scale * Q K^T - LSE)  (recomputed from the saved LSE, never stored)
+//   dV = P^T dO,   dP = dO V^T,   dS = P * (dP - D)  with D_i = dO_i . O_i,
+//   dQ = scale * dS K,   dK = scale * dS^T Q.
+// The pages name the backward pass and its recomputation of the attention
+// matrix from the saved statistics ("FlashAttention：把注意力从公式写成数据流",
+// section "用实验验证而不是背诵结论"; "[2205.14135] FlashAttention: Fast and
+// Memory-Efficient Exact Attention with IO-Awareness", section
+// "三、FLOPs（計算能力）並非 Speedup 的主因素"); the formulas are the chain rule
+// of the forward's definition.
+//
+// Layout (one CTA per 128-key block of one (b, h); it walks the query tiles that
+// can see its keys):
+//  * warp 0 (one lane): TMA loads of K_j and V_j once, then Q_i and dO_i per
+//    query tile (kStages slots);
+//  * warp 1 (one lane): the five tcgen05 MMAs of a tile --
+//      S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T     (M = 128 keys, N = 128 queries)
+//      dV  += P^T dO_i    and  dK  += dS^T Q_i       (A = P^T / dS^T from TMEM)
+//      dQ_i = dS K_j                                  (A = dS^T from shared memory,
+//                                                      MN-major: M = queries)
+//    dV and dK stay in TMEM for the whole CTA;
+//  * warps 4-7: one thread per key row (TMEM lane): P^T and dS^T from S^T and
+//    dP^T (exp2 domain, masks), written back to TMEM as bf16 over the columns
+//    just read and, for dS^T, to shared memory; then each thread reads one
+//    query row of dQ_i and adds it into the fp32 dQ accumulator in global
+//    memory (vector atomic adds: several key blocks update each query row);
+//    finally dV and scale * dK go to global memory as bf16.
+// Every mbarrier wait is bounded (as in the forward kernel); a wait that runs
+// out records FA_ERR_DEVICE_TIMEOUT and the CTA winds down.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdProducerWarp = 0;
+constexpr int kBwdMmaWarp = 1;
+constexpr int kBwdComputeWarp0 = 4;     // warps 4..7 own TMEM lane quadrants 0..3
+constexpr uint32_t kBwdBarCompute = 6;  // named barrier over the 4 compute warps
+
+struct BwdParams {
+    const float* lse;           // [B,H,Nq] the forward's LSE (natural log; -inf: no visible key)
+    const float* dsum;          // [B,H,Nq] D_i = dO_i . O_i (fa_bwd_pre_kernel)
+    float* dq_acc;              // [B,H,Nq,D] fp32 accumulator, zero on entry
+    __nv_bfloat16* dk;          // [B,H,Nk,D]
+    __nv_bfloat16* dv;          // [B,H,Nk,D]
+    const int32_t* key_lens;    // [B] or nullptr
+    int B, H, Nq, Nk;
+    float scale;                // softmax scale
+    float scale_log2;           // scale * log2(e)
+    int causal;
+    unsigned long long wait_limit;
+};
+
+template <int D>
+struct BwdCfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kStages = (D == 64) ? 2 : 1;                // Q / dO slots
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kTileBytes;
+    static constexpr int kQOff = kVOff + kTileBytes;                  // [stage]
+    static constexpr int kDOOff = kQOff + kStages * kTileBytes;       // [stage]
+    static constexpr int kDSOff = kDOOff + kStages * kTileBytes;      // dS^T: 2 boxes of 64 queries
+    static constexpr int kRowOff = kDSOff + 2 * kSwizzleBoxBytes;     // [2][lse2 x128 | D x128] fp32
+    static constexpr int kBarOff = kRowOff + 2 * 256 * 4;
+    // barriers: kv_full, q_full[S], q_empty[S], s_full, p_full, dq_full, s_free, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 5;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+    static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
+    // TMEM columns: S^T (then P^T as bf16, then dQ) at 0; dP^T (then dS^T) at 128;
+    // dV at 256; dK at 256 + D.
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static_assert(kColDK + D <= 512, "TMEM columns");
+    // Instruction descriptors (kind::f16, D = f32, A = B = bf16, M = 128):
+    //   S^T, dP^T: A K-major, B K-major, N = 128 (queries);
+    //   dV, dK:    A from TMEM, B MN-major (dO / Q rows are queries), N = D;
+    //   dQ:        A MN-major (dS^T in shared memory), B MN-major (K), N = D.
+    static constexpr uint32_t kIdescST = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
+                                         ((128u >> 3) << 17) | ((128u >> 4) << 24);
+    static constexpr uint32_t kIdescKV = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                         (((uint32_t)D >> 3) << 17) | ((128u >> 4) << 24);
+    static constexpr uint32_t kIdescQ = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                        (((uint32_t)D >> 3) << 17) | ((128u >> 4) << 24);
+};
+
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Waits for asynchronous work that completes on its own (copies already issued,
+// MMAs already issued) -- even after another role gave up -- so that nothing is
+// still writing shared memory or TMEM when the CTA releases them.  Bounded.
+__device__ __forceinline__ void wait_own_work(uint32_t bar, uint32_t parity, unsigned long long limit) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if ((unsigned long long)(clock64() - t0) > limit) break;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_base = smem_addr(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* const base_ptr = smem_raw + (base - raw_base);
+
+    auto bar = [&](int i) { return base + C::kBarOff + 8u * (uint32_t)i; };
+    const uint32_t bar_kv = bar(0);
+    auto bar_q_full = [&](int s) { return bar(1 + s); };
+    auto bar_q_empty = [&](int s) { return bar(1 + C::kStages + s); };
+    const uint32_t bar_s_full = bar(1 + 2 * C::kStages);
+    const uint32_t bar_p_full = bar(2 + 2 * C::kStages);
+    const uint32_t bar_dq_full = bar(3 + 2 * C::kStages);
+    const uint32_t bar_s_free = bar(4 + 2 * C::kStages);
+    const uint32_t bar_drain = bar(5 + 2 * C::kStages);
+    uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
+    volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
+    float* const rows = reinterpret_cast<float*>(base_ptr + C::kRowOff);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int k0 = (int)blockIdx.x * 128;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const size_t bh = (size_t)b * p.H + h;
+    int kl = p.Nk;
+    if (p.key_lens != nullptr) {
+        kl = p.key_lens[b];
+        kl = kl < 0 ? 0 : (kl > p.Nk ? p.Nk : kl);
+    }
+    const int off = p.Nk - p.Nq;   // key j visible to query i iff j <= i + off (causal)
+    const int num_m = (p.Nq + 127) / 128;
+    // the first query that can see key k0 is k0 - off (causal); all queries otherwise
+    int i_lo = 0;
+    if (p.causal) {
+        const long long f = (long long)k0 - off;
+        i_lo = f <= 0 ? 0 : (int)(f / 128 < num_m ? f / 128 : num_m);
+    }
+    const int n_t = (k0 < kl && i_lo < num_m) ? num_m - i_lo : 0;
+
+    if (warp == kBwdProducerWarp && lane == 0) {
+        mbar_init(bar_kv, 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(bar_q_full(s), 1);
+            mbar_init(bar_q_empty(s), 1);
+        }
+        mbar_init(bar_s_full, 1);
+        mbar_init(bar_p_full, 4);    // one arrival per compute warp
+        mbar_init(bar_dq_full, 1);
+        mbar_init(bar_s_free, 4);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_do);
+    }
+    if (warp == kBwdMmaWarp) {
+        tmem_alloc(smem_addr(tmem_holder), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == kBwdProducerWarp) {
+        // ============================================================ TMA producer
+        if (lane == 0 && n_t > 0) {
+            const uint64_t pol_keep = policy_evict_last();
+            mbar_arrive_expect_tx(bar_kv, 2u * (uint32_t)C::kTileBytes);
+            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                tma_load_4d(base + C::kKOff + bx * kSwizzleBoxBytes, &tm_k, bar_kv, bx * 64, k0, h, b,
+                            policy_evict_first());
+                tma_load_4d(base + C::kVOff + bx * kSwizzleBoxBytes, &tm_v, bar_kv, bx * 64, k0, h, b,
+                            policy_evict_first());
+            }
+            bool ok = true;
+            int t = 0;
+            for (; t < n_t; ++t) {
+                const int s = t % C::kStages;
+                ok = wait_bounded(bar_q_empty(s), (uint32_t)(((t / C::kStages) & 1) ^ 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_q_full(s), 2u * (uint32_t)C::kTileBytes);
+                const int q0 = (i_lo + t) * 128;
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_4d(base + C::kQOff + s * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_q, bar_q_full(s),
+                                bx * 64, q0, h, b, pol_keep);
+                    tma_load_4d(base + C::kDOOff + s * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_do,
+                                bar_q_full(s), bx * 64, q0, h, b, pol_keep);
+                }
+            }
+            // wind down: every copy issued lands before the CTA exits
+            wait_own_work(bar_kv, 0, p.wait_limit);
+            if (!ok)
+                for (int c2 = (t > C::kStages ? t - C::kStages : 0); c2 < t; ++c2)
+                    wait_own_work(bar_q_full(c2 % C::kStages), (uint32_t)((c2 / C::kStages) & 1), p.wait_limit);
+        }
+        __syncwarp();
+    } else if (warp == kBwdMmaWarp) {
+        // ============================================================ MMA issuer
+        if (lane == 0 && n_t > 0) {
+            bool ok = wait_bounded(bar_kv, 0, abort_flag, p.wait_limit);
+            const uint32_t k_s = base + C::kKOff, v_s = base + C::kVOff, ds_s = base + C::kDSOff;
+            for (int t = 0; t < n_t && ok; ++t) {
+                const int s = t % C::kStages;
+                ok = wait_bounded(bar_q_full(s), (uint32_t)((t / C::kStages) & 1), abort_flag, p.wait_limit);
+                // the previous tile's dQ has been read out of the S columns
+                if (ok && t > 0) ok = wait_bounded(bar_s_free, (uint32_t)((t - 1) & 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t q_s = base + C::kQOff + s * C::kTileBytes;
+                const uint32_t do_s = base + C::kDOOff + s * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
+                    const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
+                    umma_ss(tmem + C::kColS, smem_desc_sw128(k_s + koff, 16, 1024), smem_desc_sw128(q_s + koff, 16, 1024),
+                            C::kIdescST, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
+                    const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
+                    umma_ss(tmem + C::kColDP, smem_desc_sw128(v_s + koff, 16, 1024),
+                            smem_desc_sw128(do_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar_s_full);
+                ok = wait_bounded(bar_p_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 128 / 16; ++kk) {   // dV += P^T dO: 16 queries per step
+                    umma_ts(tmem + C::kColDV, tmem + C::kColS + (uint32_t)(kk * 8),
+                            smem_desc_sw128(do_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 128 / 16; ++kk) {   // dK += dS^T Q
+                    umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(kk * 8),
+                            smem_desc_sw128(q_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar_q_empty(s));   // Q_i and dO_i are no longer read
+#pragma unroll
+                for (int kk = 0; kk < 128 / 16; ++kk) {   // dQ = dS K: 16 keys per step
+                    umma_ss(tmem + C::kColS, smem_desc_sw128(ds_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024),
+                            smem_desc_sw128(k_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescQ,
+                            kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar_dq_full);
+            }
+            // every MMA issued has completed before TMEM is released (also after a give-up)
+            umma_commit(bar_drain);
+            wait_own_work(bar_drain, 0, p.wait_limit);
+        }
+        __syncwarp();
+    } else if (warp >= kBwdComputeWarp0) {
+        // ============================================================ P, dS, dQ, and the epilogue
+        const int qd = warp - kBwdComputeWarp0;   // TMEM lane quadrant (warp % 4)
+        const int r = qd * 32 + lane;             // key row in the block (S^T lanes) / query row (dQ lanes)
+        const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+        const int k = k0 + r;
+        const bool key_ok = k < kl;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int t = 0; t < n_t; ++t) {
+            const int i0 = (i_lo + t) * 128;
+            float* const rb = rows + (t & 1) * 256;
+            {
+                // this thread's query row of the tile: its LSE (log2 units; +inf
+                // when the row sees no key, or lies past N_q) and D
+                const int q = i0 + r;
+                float l2 = INFINITY, dd = 0.f;
+                if (q < p.Nq) {
+                    const float L = p.lse[bh * (size_t)p.Nq + q];
+                    l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
+                    dd = p.dsum[bh * (size_t)p.Nq + q];
+                }
+                rb[r] = l2;
+                rb[128 + r] = dd;
+            }
+            // all four warps wrote the tile's row data; leave together if any gave up
+            if (named_bar_or(kBwdBarCompute, 128, !ok)) break;
+            bool good = wait_bounded(bar_s_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
+            if (!__all_sync(0xffffffffu, good)) {
+                ok = false;
+                continue;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {   // queries 32cb .. 32cb+31
+                uint32_t su[32], du[32];
+                tmem_ld32(tmem + lane_off + C::kColS + 32u * cb, su);
+                tmem_ld32(tmem + lane_off + C::kColDP + 32u * cb, du);
+                tmem_wait_ld();
+                uint32_t pw[16], dw[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    reg_after_wait(su[e]);
+                    reg_after_wait(su[e + 1]);
+                    reg_after_wait(du[e]);
+                    reg_after_wait(du[e + 1]);
+                    const int qa = i0 + 32 * cb + e;
+                    const bool v0 = key_ok && (!p.causal || k <= qa + off);
+                    const bool v1 = key_ok && (!p.causal || k <= qa + 1 + off);
+                    const float p0 = v0 ? ex2_approx(__uint_as_float(su[e]) * c - rb[32 * cb + e]) : 0.f;
+                    const float p1 = v1 ? ex2_approx(__uint_as_float(su[e + 1]) * c - rb[32 * cb + e + 1]) : 0.f;
+                    const float d0 = p0 * (__uint_as_float(du[e]) - rb[128 + 32 * cb + e]);
+                    const float d1 = p1 * (__uint_as_float(du[e + 1]) - rb[128 + 32 * cb + e + 1]);
+                    pw[e >> 1] = pack_bf16x2(p0, p1);
+                    dw[e >> 1] = pack_bf16x2(d0, d1);
+                }
+                // P^T over S^T's columns 16cb.., dS^T over dP^T's (both already read)
+                tmem_st16(tmem + lane_off + C::kColS + 16u * cb, pw);
+                tmem_st16(tmem + lane_off + C::kColDP + 16u * cb, dw);
+                // dS^T row r into shared memory: box cb/2 holds queries 64(cb/2)..+63 as
+                // 128-byte rows, 16-byte chunk cc at swizzled position cc ^ (r % 8)
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4) {
+                    const int cc = (cb & 1) * 4 + t4;
+                    const uint32_t a = base + C::kDSOff + (uint32_t)((cb >> 1) * kSwizzleBoxBytes + r * 128 +
+                                                                     ((cc ^ (r & 7)) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(dw[4 * t4]),
+                                 "r"(dw[4 * t4 + 1]), "r"(dw[4 * t4 + 2]), "r"(dw[4 * t4 + 3])
+                                 : "memory");
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();   // dS^T visible to the tensor core
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p_full);
+            // dQ_i (TMEM lane = query row i0 + r) into the fp32 accumulator
+            good = wait_bounded(bar_dq_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
+            if (!__all_sync(0xffffffffu, good)) {
+                ok = false;
+                continue;
+            }
+            tc_fence_after();
+            const int q = i0 + r;
+#pragma unroll 1
+            for (int c2 = 0; c2 < D / 32; ++c2) {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_off + C::kColS + 32u * c2, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) reg_after_wait(u[i]);
+                if (q < p.Nq) {
+                    float* dst = p.dq_acc + (bh * (size_t)p.Nq + q) * D + 32 * c2;
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        red_add_v4(dst + 4 * v4, __uint_as_float(u[4 * v4]), __uint_as_float(u[4 * v4 + 1]),
+                                   __uint_as_float(u[4 * v4 + 2]), __uint_as_float(u[4 * v4 + 3]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s_free);
+        }
+        // ------------------------------------------------------------ dV, dK -> bf16
+        bool have = n_t > 0;
+        if (have && ok) {
+            const bool good = wait_bounded(bar_drain, 0, abort_flag, p.wait_limit);
+            ok = __all_sync(0xffffffffu, good);
+            if (ok) tc_fence_after();
+        }
+        // tcgen05.ld is warp-collective: every lane loads (ok is warp-uniform), and
+        // only the stores are limited to keys < N_k
+        if (ok) {
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* const out = which == 0 ? p.dv : p.dk;
+                const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
+                const float f = which == 0 ? 1.f : p.scale;
+#pragma unroll 1
+                for (int c2 = 0; c2 < D / 32; ++c2) {
+                    uint32_t u[32];
+                    if (have) {
+                        tmem_ld32(tmem + lane_off + col + 32u * c2, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) reg_after_wait(u[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = 0u;
+                    }
+                    if (k >= p.Nk) continue;
+                    uint4* dst = reinterpret_cast<uint4*>(out + (bh * (size_t)p.Nk + k) * D + 32 * c2);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 w4;
+                        w4.x = pack_bf16x2(__uint_as_float(u[8 * v4]) * f, __uint_as_float(u[8 * v4 + 1]) * f);
+                        w4.y = pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * f, __uint_as_float(u[8 * v4 + 3]) * f);
+                        w4.z = pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * f, __uint_as_float(u[8 * v4 + 5]) * f);
+                        w4.w = pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * f, __uint_as_float(u[8 * v4 + 7]) * f);
+                        dst[v4] = w4;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == kBwdMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// D_i = dO_i . O_i (fp32) for every query row, and the dQ accumulator row zeroed.
+// One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                      float* __restrict__ dsum, float* __restrict__ dq_acc, long long rows) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int kPer = D / 32;   // consecutive columns per lane
+    const __nv_bfloat16* po = o + row * D + lane * kPer;
+    const __nv_bfloat16* pd = dout + row * D + lane * kPer;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc = fmaf(__bfloat162float(po[i]), __bfloat162float(pd[i]), acc);
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+    if (lane == 0) dsum[row] = acc;
+    float* z = dq_acc + row * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) z[i] = 0.f;
+}
+
+// dQ = bf16(scale * dQ accumulator), 8 elements per thread.
+__global__ void __launch_bounds__(256)
+    fa_bwd_post_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, float scale, long long n8) {
+    const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
+    const float4 b2 = reinterpret_cast<const float4*>(dq_acc)[2 * i + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x * scale, a.y * scale);
+    w.y = pack_bf16x2(a.z * scale, a.w * scale);
+    w.z = pack_bf16x2(b2.x * scale, b2.y * scale);
+    w.w = pack_bf16x2(b2.z * scale, b2.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = w;
+}
+
+}  // namespace fa

@@ -10,7 +10,7 @@ Recipe (stated once, used everywhere):
 * generator: numpy's ``Philox`` bit generator (Philox4x64-10, Salmon et al.,
   "Parallel random numbers: as easy as 1, 2, 3", SC'11), one independent stream
   per tensor, keyed by ``seed * 16 + tensor_id`` with tensor_id Q=0, K=1, V=2,
-  key_lens=3;
+  key_lens=3, dO=4 (the backward pass's upstream gradient);
 * values: ``standard_normal`` in float32 times sigma (sigma = 1 or 0.5, both
   exact in float32), rounded to bf16 with round-to-nearest-even;
 * key lengths: integers uniform on [lo, hi] inclusive, one per sequence,
@@ -29,6 +29,7 @@ import math
 import numpy as np
 
 TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_KEYLEN = 0, 1, 2, 3
+TENSOR_DO = 4   # upstream gradient dL/dO for the backward pass
 
 
 @dataclasses.dataclass(frozen=True)
