@@ -284,6 +284,62 @@ def fp8_table(steps, warmup, device, peak_bf16_tflops):
     return out
 
 
+def time_bwd(w, x, steps, warmup, device):
+    """Mean per-call device time (ms) of fa_bwd (its four launches) on resident inputs,
+    the forward's O and LSE computed once beforehand; L2 flushed between calls."""
+    import torch
+    from io_aware_exact_24_b200 import fa_bwd, fa_bwd_workspace_size, fa_fwd
+    from io_aware_exact_24_b200.inputs import TENSOR_DO, normal_bf16
+    q, k, v, kl = upload(x, device)
+    do = torch.from_numpy(normal_bf16((w.B, w.H, w.Nq, w.d), w.seed, TENSOR_DO, w.sigma).view(np.int16)).to(
+        device).view(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    fa_fwd(q, k, v, o, lse, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl, stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nb = fa_bwd_workspace_size(w.B, w.H, w.Nq, w.d)
+    ws = torch.empty(nb, dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def launch():
+        fa_bwd(q, k, v, o, lse, do, dq, dk, dv, w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, kl, ws, nb,
+               stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for st, en in ev:
+        flush.zero_()
+        st.record(stream)
+        launch()
+        en.record(stream)
+    torch.cuda.synchronize()
+    per = [st.elapsed_time(en) for st, en in ev]
+    del q, k, v, o, lse, do, dq, dk, dv, ws, flush
+    return float(np.mean(per))
+
+
+def bwd_table(steps, warmup, device, peak_tflops):
+    """Backward pass (fa_bwd): FLOPs = 2.5 x the forward's (five products of the
+    forward's size instead of two), tensor roofline against the measured bf16 peak."""
+    out = {}
+    for name in ("causal_8000_d128", "long_16k_d64"):
+        w = WORKLOADS[name]
+        ms = time_bwd(w, make_inputs(w), steps, warmup, device)
+        flop = 2.5 * w.flop
+        tf = flop / (ms / 1000.0) / 1e12
+        out[name] = {"entry": "fa_bwd", "ms": ms, "tflops": tf,
+                     "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tflops,
+                                  "unit": "TFLOP/s", "frac": tf / peak_tflops},
+                     "flop": "2.5 x (4*B*H*Nq*Nk*d, causal halved)",
+                     "config": config_of(w, "flushed between timed calls", "single GPU")}
+    return out
+
+
 def varlen_table(steps, warmup, device, peak_tflops):
     """Packed variable-length batch with the BERT-shaped lengths of bert_padded_512
     (each sequence's queries and keys = its key length), against the padded
@@ -511,6 +567,8 @@ def main():
                     help="time only the split-KV forward on this decode workload (profiling runs)")
     ap.add_argument("--fp8-only", action="store_true",
                     help="time only the E4M3 forward on causal_8000_d128 (profiling runs)")
+    ap.add_argument("--bwd-only", default=None, choices=["causal_8000_d128", "long_16k_d64"],
+                    help="time only the backward pass on this workload (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -542,6 +600,13 @@ def main():
                                        "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                        "frac": gbs / float(peaks["hbm_gbs"])},
                           "config": config_of(w, "flushed between timed launches", "single GPU")}),
+              flush=True)
+        return 0
+    if args.bwd_only:
+        w = WORKLOADS[args.bwd_only]
+        ms = time_bwd(w, make_inputs(w), args.steps, args.warmup, device)
+        print(json.dumps({"backward": {args.bwd_only: {"ms": ms,
+                                                       "tflops": 2.5 * w.flop / (ms / 1000.0) / 1e12}}}),
               flush=True)
         return 0
     if args.fp8_only:
@@ -601,6 +666,7 @@ def main():
         line["sliding_window"] = window_table(args.steps, args.warmup, device, peak)
         line["varlen"] = varlen_table(args.steps, args.warmup, device, peak)
         line["fp8"] = fp8_table(args.steps, args.warmup, device, peak)
+        line["backward"] = bwd_table(args.steps, args.warmup, device, peak)
         cpu_s = float(os.environ.get("FA_CPU_BASELINE_SECONDS", "15"))
         rate, n, t, cores = oracle_sample_rate(w, x, cpu_s)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",

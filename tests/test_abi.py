@@ -314,3 +314,52 @@ def test_fp8_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert fp8_call() == binding.FA_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- backward entry point
+
+def bwd_call(ws_bytes=None, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, do=P, dq=P, dk=P, dv=P, B=1, H=2, Nq=8, Nk=8, d=64,
+             scale=0.125, causal=1, key_lens=None, ws=P)
+    a.update(kw)
+    need = binding.fa_bwd_workspace_size(a["B"], a["H"], a["Nq"], a["d"])
+    return binding.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"],
+                          a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                          a["key_lens"], a["ws"], need if ws_bytes is None else ws_bytes, stream=0,
+                          check=False)
+
+
+def test_bwd_workspace_size(lib):
+    # D [B,H,N_q] fp32 then the fp32 dQ accumulator, each rounded up to 256 bytes
+    assert binding.fa_bwd_workspace_size(2, 3, 100, 64) == 2560 + 153600
+    assert binding.fa_bwd_workspace_size(1, 1, 1, 128) == 256 + 512
+    assert binding.fa_bwd_workspace_size(1, 1, 1, 96) == 0
+    assert binding.fa_bwd_workspace_size(-1, 1, 1, 64) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(do=None), binding.FA_ERR_INVALID_ARG),
+    (dict(dq=None), binding.FA_ERR_INVALID_ARG),
+    (dict(dk=None), binding.FA_ERR_INVALID_ARG),
+    (dict(dv=None), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=None), binding.FA_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=P + 128), binding.FA_ERR_MISALIGNED),
+    (dict(do=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(dk=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(q=P + 8), binding.FA_ERR_MISALIGNED),
+    (dict(B=0, q=None, do=None), binding.FA_OK),
+    (dict(Nq=0, q=None, o=None, lse=None, do=None, dq=None, dk=None), binding.FA_ERR_INVALID_ARG),
+])
+def test_bwd_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert bwd_call(**kw) == code
+
+
+def test_bwd_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert bwd_call() == binding.FA_ERR_NO_DEVICE
