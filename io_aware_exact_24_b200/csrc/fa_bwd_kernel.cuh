@@ -22,12 +22,13 @@
 //      dQ_i = dS K_j                                  (A = dS^T from shared memory,
 //                                                      MN-major: M = queries)
 //    dV and dK stay in TMEM for the whole CTA;
-//  * warps 4-7: one thread per key row (TMEM lane): P^T and dS^T from S^T and
-//    dP^T (exp2 domain, masks), written back to TMEM as bf16 over the columns
-//    just read and, for dS^T, to shared memory; then each thread reads one
-//    query row of dQ_i and adds it into the fp32 dQ accumulator in global
-//    memory (vector atomic adds: several key blocks update each query row);
-//    finally dV and scale * dK go to global memory as bf16.
+//  * warps 4-11, two per TMEM lane quadrant, each thread one key row and half
+//    of the columns: P^T and dS^T from S^T and dP^T (exp2 domain, masks),
+//    written back to TMEM as bf16 over the columns just read and, for dS^T, to
+//    shared memory; then each thread reads half of one query row of dQ_i and
+//    adds it into the fp32 dQ accumulator in global memory (vector atomic adds:
+//    several key blocks update each query row); finally dV and scale * dK go to
+//    global memory as bf16.
 // Every mbarrier wait is bounded (as in the forward kernel); a wait that runs
 // out records FA_ERR_DEVICE_TIMEOUT and the CTA winds down.
 #pragma once
@@ -36,11 +37,12 @@
 
 namespace fa {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 384;
 constexpr int kBwdProducerWarp = 0;
 constexpr int kBwdMmaWarp = 1;
-constexpr int kBwdComputeWarp0 = 4;     // warps 4..7 own TMEM lane quadrants 0..3
-constexpr uint32_t kBwdBarCompute = 6;  // named barrier over the 4 compute warps
+constexpr int kBwdComputeWarp0 = 4;     // warps 4..11: two per TMEM lane quadrant (warp % 4)
+constexpr int kBwdComputeWarps = 8;
+constexpr uint32_t kBwdBarCompute = 6;  // named barrier over the 8 compute warps
 
 struct BwdParams {
     const float* lse;           // [B,H,Nq] the forward's LSE (natural log; -inf: no visible key)
@@ -75,7 +77,9 @@ struct BwdCfg {
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
     // TMEM columns: S^T (then P^T as bf16, then dQ) at 0; dP^T (then dS^T) at 128;
-    // dV at 256; dK at 256 + D.
+    // dV at 256; dK at 256 + D.  P^T of queries 0-63 sits at columns 0-31 and of
+    // queries 64-127 at 64-95 (dS^T likewise from 128), so each compute warp
+    // overwrites only columns it has itself read.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
     static_assert(kColDK + D <= 512, "TMEM columns");
     // Instruction descriptors (kind::f16, D = f32, A = B = bf16, M = 128):
@@ -156,9 +160,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(bar_q_empty(s), 1);
         }
         mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, 4);    // one arrival per compute warp
+        mbar_init(bar_p_full, kBwdComputeWarps);    // one arrival per compute warp
         mbar_init(bar_dq_full, 1);
-        mbar_init(bar_s_free, 4);
+        mbar_init(bar_s_free, kBwdComputeWarps);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -241,13 +245,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 128 / 16; ++kk) {   // dV += P^T dO: 16 queries per step
-                    umma_ts(tmem + C::kColDV, tmem + C::kColS + (uint32_t)(kk * 8),
+                    // P^T of queries 16kk.. at column 8kk (first 64 queries) or 8kk + 32
+                    umma_ts(tmem + C::kColDV, tmem + C::kColS + (uint32_t)(kk * 8 + 32 * (kk / 4)),
                             smem_desc_sw128(do_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 128 / 16; ++kk) {   // dK += dS^T Q
-                    umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(kk * 8),
+                    umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(kk * 8 + 32 * (kk / 4)),
                             smem_desc_sw128(q_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -267,7 +272,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncwarp();
     } else if (warp >= kBwdComputeWarp0) {
         // ============================================================ P, dS, dQ, and the epilogue
-        const int qd = warp - kBwdComputeWarp0;   // TMEM lane quadrant (warp % 4)
+        const int qd = warp & 3;                  // TMEM lane quadrant
+        const int g = (warp - kBwdComputeWarp0) >> 2;   // which half of the columns this warp takes
         const int r = qd * 32 + lane;             // key row in the block (S^T lanes) / query row (dQ lanes)
         const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
         const int k = k0 + r;
@@ -287,11 +293,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
                     dd = p.dsum[bh * (size_t)p.Nq + q];
                 }
-                rb[r] = l2;
-                rb[128 + r] = dd;
+                if (g == 0) {
+                    rb[r] = l2;
+                    rb[128 + r] = dd;
+                }
             }
             // all four warps wrote the tile's row data; leave together if any gave up
-            if (named_bar_or(kBwdBarCompute, 128, !ok)) break;
+            if (named_bar_or(kBwdBarCompute, 32 * kBwdComputeWarps, !ok)) break;
             bool good = wait_bounded(bar_s_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
             if (!__all_sync(0xffffffffu, good)) {
                 ok = false;
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {   // queries 32cb .. 32cb+31
+            for (int cb = 2 * g; cb < 2 * g + 2; ++cb) {   // queries 32cb .. 32cb+31
                 uint32_t su[32], du[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32u * cb, su);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32u * cb, du);
@@ -321,9 +329,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pw[e >> 1] = pack_bf16x2(p0, p1);
                     dw[e >> 1] = pack_bf16x2(d0, d1);
                 }
-                // P^T over S^T's columns 16cb.., dS^T over dP^T's (both already read)
-                tmem_st16(tmem + lane_off + C::kColS + 16u * cb, pw);
-                tmem_st16(tmem + lane_off + C::kColDP + 16u * cb, dw);
+                // P^T over S^T's columns 16cb + 32g.., dS^T over dP^T's: inside the 64
+                // columns this warp has read (the other warp of the quadrant reads
+                // the other 64), and after this warp read them
+                tmem_st16(tmem + lane_off + C::kColS + 16u * cb + 32u * g, pw);
+                tmem_st16(tmem + lane_off + C::kColDP + 16u * cb + 32u * g, dw);
                 // dS^T row r into shared memory: box cb/2 holds queries 64(cb/2)..+63 as
                 // 128-byte rows, 16-byte chunk cc at swizzled position cc ^ (r % 8)
 #pragma unroll
@@ -350,7 +360,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             const int q = i0 + r;
 #pragma unroll 1
-            for (int c2 = 0; c2 < D / 32; ++c2) {
+            for (int c2 = g * (D / 64); c2 < (g + 1) * (D / 64); ++c2) {   // this warp's half of dQ
                 uint32_t u[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32u * c2, u);
                 tmem_wait_ld();
@@ -384,7 +394,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
                 const float f = which == 0 ? 1.f : p.scale;
 #pragma unroll 1
-                for (int c2 = 0; c2 < D / 32; ++c2) {
+                for (int c2 = g * (D / 64); c2 < (g + 1) * (D / 64); ++c2) {
                     uint32_t u[32];
                     if (have) {
                         tmem_ld32(tmem + lane_off + col + 32u * c2, u);
