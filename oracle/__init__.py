@@ -59,31 +59,42 @@ def _load():
             build()
             lib = ctypes.CDLL(_LIB_PATH)
             i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            f64 = ctypes.c_double
             vp = ctypes.c_void_p
             lib.attn_ref_fp64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
-                                          f32, i32, vp, vp, vp]
+                                          f64, i32, vp, vp, vp]
             lib.attn_ref_fp64.restype = i32
             lib.attn_ref_fp64_window.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
-                                                 f32, i32, i64, vp, vp, vp]
+                                                 f64, i32, i64, vp, vp, vp]
             lib.attn_ref_fp64_window.restype = i32
             lib.attn_ref_fp64_bias.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
-                                               f32, i32, i64, vp, vp, vp, vp]
+                                               f64, i32, i64, vp, vp, vp, vp]
             lib.attn_ref_fp64_bias.restype = i32
+            lib.attn_ref_fp64_bias_table.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                                     f64, i32, i64, vp, i64, vp, vp, vp]
+            lib.attn_ref_fp64_bias_table.restype = i32
             lib.attn_ref_fp64_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
-                                               i64, f32, i32, vp, i64, vp, vp]
+                                               i64, f64, i32, vp, i64, vp, vp]
             lib.attn_ref_fp64_rows.restype = i32
             lib.attn_online_fp64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
                                              i64, f32, i32, i64, vp, vp]
             lib.attn_online_fp64.restype = i32
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i32
+            lib.oracle_set_num_threads.argtypes = [i32]
+            lib.oracle_set_num_threads.restype = None
             _lib = lib
     return _lib
 
 
 def num_threads() -> int:
-    """OpenMP threads the oracle uses (set OMP_NUM_THREADS to change)."""
+    """OpenMP threads the oracle uses (set OMP_NUM_THREADS, or set_num_threads, to change)."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Use n OpenMP threads in the following oracle calls (n >= 1)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _ptr(a):
@@ -107,13 +118,19 @@ def _check(q, k, v, key_lens):
 
 
 def attn_ref(q, k, v, scale, causal=False, key_lens=None, return_p=False):
-    """Plain definition.  Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq][, P])."""
+    """Plain definition.  Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq][, P]).
+    ``scale`` is rounded to fp32 first: it is the fp32 value the library receives."""
+    return _attn_ref_f64scale(q, k, v, float(np.float32(scale)), causal, key_lens, return_p)
+
+
+def _attn_ref_f64scale(q, k, v, scale, causal=False, key_lens=None, return_p=False):
+    """attn_ref with ``scale`` taken as the fp64 value given (no rounding)."""
     q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
     o = np.empty((B, H, Nq, d), np.float64)
     lse = np.empty((B, H, Nq), np.float64)
     p = np.empty((B, H, Nq, Nk), np.float64) if return_p else None
     rc = _load().attn_ref_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
-                               Nq, Nk, d, float(np.float32(scale)), int(bool(causal)),
+                               Nq, Nk, d, float(scale), int(bool(causal)),
                                _ptr(o), _ptr(lse), _ptr(p))
     if rc != 0:
         raise RuntimeError(f"attn_ref_fp64 failed ({rc})")
@@ -151,6 +168,26 @@ def attn_ref_bias(q, k, v, scale, slopes, causal=False, key_lens=None, window_le
     return o, lse
 
 
+def attn_ref_bias_table(q, k, v, scale, table, causal=False, key_lens=None, window_left=-1):
+    """Plain definition with a custom positional bias: table fp32 [H, 2R+1] adds
+    table[h, clamp(j - (i + Nk - Nq), -R, R) + R] to the score of query i and key j
+    (natural-log units, after the scale), optionally with a sliding window.
+    Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq])."""
+    q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
+    tb = np.ascontiguousarray(table, dtype=np.float32)
+    if tb.ndim != 2 or tb.shape[0] != H or tb.shape[1] % 2 != 1:
+        raise ValueError("table must be fp32 [H, 2R+1]")
+    R = (tb.shape[1] - 1) // 2
+    o = np.empty((B, H, Nq, d), np.float64)
+    lse = np.empty((B, H, Nq), np.float64)
+    rc = _load().attn_ref_fp64_bias_table(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H, Nq,
+                                          Nk, d, float(np.float32(scale)), int(bool(causal)),
+                                          int(window_left), _ptr(tb), R, _ptr(o), _ptr(lse), None)
+    if rc != 0:
+        raise RuntimeError(f"attn_ref_fp64_bias_table failed ({rc})")
+    return o, lse
+
+
 def attn_ref_varlen(q, k, v, cu_q, cu_k, scale, causal=False):
     """Packed variable-length batches: q [Tq,H,d], k/v [Tk,H,d] bf16 bits, cu_q/cu_k
     int [B+1].  Each sequence is an independent problem, evaluated with attn_ref on
@@ -175,13 +212,19 @@ def attn_ref_varlen(q, k, v, cu_q, cu_k, scale, causal=False):
 
 
 def attn_ref_rows(q, k, v, scale, row_ids, causal=False, key_lens=None):
-    """Definition on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n])."""
+    """Definition on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n]).
+    ``scale`` is rounded to fp32 first, as in attn_ref."""
+    return _attn_ref_rows_f64scale(q, k, v, float(np.float32(scale)), row_ids, causal, key_lens)
+
+
+def _attn_ref_rows_f64scale(q, k, v, scale, row_ids, causal=False, key_lens=None):
+    """attn_ref_rows with ``scale`` taken as the fp64 value given."""
     q, k, v, key_lens, B, H, Nq, Nk, d = _check(q, k, v, key_lens)
     rows = np.ascontiguousarray(row_ids, dtype=np.int64)
     o = np.empty((rows.size, d), np.float64)
     lse = np.empty((rows.size,), np.float64)
     rc = _load().attn_ref_fp64_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(key_lens), B, H,
-                                    Nq, Nk, d, float(np.float32(scale)),
+                                    Nq, Nk, d, float(scale),
                                     int(bool(causal)), _ptr(rows), rows.size,
                                     _ptr(o), _ptr(lse))
     if rc != 0:
@@ -235,25 +278,30 @@ def e4m3_to_bf16_bits(codes) -> np.ndarray:
 
 
 def _e4m3_scale(scale, q_descale, k_descale):
-    # Reading: the three fp32 factors of the scores are folded into one fp32 scale
-    # (a relative change of at most 2^-24 in every score).
-    return float(np.float32(np.float64(scale) * np.float64(q_descale) * np.float64(k_descale)))
+    # The scores of the dequantised inputs are scale * (qd Q8)(kd K8)^T =
+    # (scale * qd * kd) * Q8 K8^T: the product of the three fp32 factors, taken
+    # exactly (in fp64, where the product of three 24-bit significands is off by
+    # at most one rounding of 2^-53), not folded into one fp32 number.
+    return float(np.float64(np.float32(scale)) * np.float64(np.float32(q_descale))
+                 * np.float64(np.float32(k_descale)))
 
 
 def attn_ref_e4m3(q8, k8, v8, scale, q_descale, k_descale, v_descale, causal=False, key_lens=None):
     """Plain definition on dequantised e4m3 inputs (uint8 codes [B,H,N,d]):
     softmax(scale * (qd Q8)(kd K8)^T) (vd V8) = vd * attn(Q8, K8, V8; scale*qd*kd).
     Returns (O fp64 [B,H,Nq,d], LSE fp64 [B,H,Nq])."""
-    o, lse = attn_ref(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8), e4m3_to_bf16_bits(v8),
-                      _e4m3_scale(scale, q_descale, k_descale), causal, key_lens)
+    o, lse = _attn_ref_f64scale(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8),
+                                e4m3_to_bf16_bits(v8), _e4m3_scale(scale, q_descale, k_descale),
+                                causal, key_lens)
     return o * np.float64(np.float32(v_descale)), lse
 
 
 def attn_ref_rows_e4m3(q8, k8, v8, scale, q_descale, k_descale, v_descale, row_ids, causal=False,
                        key_lens=None):
     """attn_ref_e4m3 on selected flat rows r=(b*H+h)*Nq+i.  Returns (O [n,d], LSE [n])."""
-    o, lse = attn_ref_rows(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8), e4m3_to_bf16_bits(v8),
-                           _e4m3_scale(scale, q_descale, k_descale), row_ids, causal, key_lens)
+    o, lse = _attn_ref_rows_f64scale(e4m3_to_bf16_bits(q8), e4m3_to_bf16_bits(k8),
+                                     e4m3_to_bf16_bits(v8), _e4m3_scale(scale, q_descale, k_descale),
+                                     row_ids, causal, key_lens)
     return o * np.float64(np.float32(v_descale)), lse
 
 

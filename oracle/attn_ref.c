@@ -31,6 +31,12 @@
  *     m_h, S_ij += -m_h * |i + (N_k - N_q) - j| on the visible entries (a
  *     linear distance penalty from the row's diagonal position, the
  *     "additive positional bias" mask variant).
+ *   - custom positional bias table (attn_ref_fp64_bias_table only): a caller's
+ *     per-head table T_h of 2R+1 values indexed by the key's position relative
+ *     to the row's diagonal position, clamped to [-R, R]:
+ *         S_ij += T_h[clamp(j - (i + N_k - N_q), -R, R) + R]
+ *     (any function of relative position within R, constant beyond it: the
+ *     general "custom positional bias" of the same section).
  *
  * Nothing here is shared with the CUDA path.  Only tests/, the package's
  * graft entry smoke check and bench.py's CPU baseline may call it.
@@ -56,6 +62,15 @@ int oracle_num_threads(void) {
     return omp_get_max_threads();
 #else
     return 1;
+#endif
+}
+
+/* Threads for the following calls (n >= 1); used to time the oracle on one core. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
 #endif
 }
 
@@ -92,9 +107,10 @@ static int64_t row_start(int64_t i, int64_t Nq, int64_t Nk, int64_t W) {
 static void one_row(const uint16_t *q_row, const uint16_t *k_head,
                     const uint16_t *v_head, int64_t Nk, int64_t d,
                     double scale, int64_t lo, int64_t lim, double slope, int64_t pos,
+                    const float *table, int64_t R,
                     double *s_row, double *p_row, double *o_row, double *lse_out) {
-    /* S_ij = scale * sum_c q_ic k_jc (- slope * |pos - j|) for valid j, -inf
-     * for masked j. */
+    /* S_ij = scale * sum_c q_ic k_jc (- slope * |pos - j|) (+ table[...]) for
+     * valid j, -inf for masked j. */
     for (int64_t j = 0; j < Nk; ++j) {
         if (j >= lo && j < lim) {
             double dot = 0.0;
@@ -102,6 +118,12 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
                 dot += bf16_bits_to_f64(q_row[c]) * bf16_bits_to_f64(k_head[j * d + c]);
             s_row[j] = scale * dot;
             if (slope != 0.0) s_row[j] -= slope * (double)llabs(pos - j);
+            if (table) {
+                int64_t r = j - pos;
+                if (r < -R) r = -R;
+                if (r > R) r = R;
+                s_row[j] += (double)table[r + R];
+            }
         } else {
             s_row[j] = -INFINITY;
         }
@@ -134,7 +156,9 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
  * Full forward.  q: bf16 bits [B,H,Nq,d]; k, v: bf16 bits [B,H,Nk,d];
  * key_lens: int32 [B] or NULL.  o: fp64 [B,H,Nq,d]; lse: fp64 [B,H,Nq].
  * p_out: NULL, or fp64 [B,H,Nq,Nk] receiving the materialised P.
- * scale is the fp32 value the GPU receives, widened to fp64.
+ * scale is a double: the bf16 callers pass the fp32 value the GPU receives,
+ * widened; the E4M3 wrapper passes the exact fp64 product of its three
+ * score factors (scale * q_descale * k_descale).
  * Returns 0, or -1 on bad sizes / allocation failure.
  */
 /*
@@ -144,28 +168,29 @@ static void one_row(const uint16_t *q_row, const uint16_t *k_head,
  */
 int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                       int64_t Nk, int64_t d, float scale, int causal,
+                       int64_t Nk, int64_t d, double scale, int causal,
                        int64_t window_left, const float *slopes, double *o, double *lse,
                        double *p_out);
 
 int attn_ref_fp64_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                         int64_t Nk, int64_t d, float scale, int causal,
+                         int64_t Nk, int64_t d, double scale, int causal,
                          int64_t window_left, double *o, double *lse, double *p_out) {
     return attn_ref_fp64_bias(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, window_left,
                               NULL, o, lse, p_out);
 }
 
 /*
- * Forward with a sliding window (window_left < 0: none) and an additive
- * positional bias (slopes: fp32 [H], one slope per head, or NULL: none).
+ * Forward with a sliding window (window_left < 0: none), a linear additive
+ * positional bias (slopes: fp32 [H], one slope per head, or NULL: none) and a
+ * custom positional bias table (table: fp32 [H, 2R+1], or NULL: none).
  */
-int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                       const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                       int64_t Nk, int64_t d, float scale, int causal,
-                       int64_t window_left, const float *slopes, double *o, double *lse,
-                       double *p_out) {
-    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0) return -1;
+static int attn_ref_general(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                            int64_t Nk, int64_t d, double scale, int causal,
+                            int64_t window_left, const float *slopes, const float *table,
+                            int64_t R, double *o, double *lse, double *p_out) {
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0 || R < 0) return -1;
     const double sc = (double)scale;
     const int64_t rows = B * H * Nq;
     int failed = 0;
@@ -185,8 +210,9 @@ int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
                 const int64_t lo = row_start(i, Nq, Nk, window_left);
                 const double slope = slopes ? (double)slopes[bh % H] : 0.0;
+                const float *tab = table ? table + (bh % H) * (2 * R + 1) : NULL;
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        lo, lim, slope, i + (Nk - Nq), s_row, p_row, o + r * d, lse + r);
+                        lo, lim, slope, i + (Nk - Nq), tab, R, s_row, p_row, o + r * d, lse + r);
                 if (p_out) memcpy(p_out + r * Nk, p_row, sizeof(double) * (size_t)Nk);
             }
         }
@@ -196,9 +222,33 @@ int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     return failed ? -1 : 0;
 }
 
+/* Forward with a sliding window and a linear additive positional bias. */
+int attn_ref_fp64_bias(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                       int64_t Nk, int64_t d, double scale, int causal,
+                       int64_t window_left, const float *slopes, double *o, double *lse,
+                       double *p_out) {
+    return attn_ref_general(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, window_left,
+                            slopes, NULL, 0, o, lse, p_out);
+}
+
+/*
+ * Forward with a sliding window and a custom positional bias table:
+ * table fp32 [H, 2R+1], R >= 0 (see the header comment).
+ */
+int attn_ref_fp64_bias_table(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
+                             int64_t Nk, int64_t d, double scale, int causal,
+                             int64_t window_left, const float *table, int64_t R, double *o,
+                             double *lse, double *p_out) {
+    if (!table) return -1;
+    return attn_ref_general(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, window_left,
+                            NULL, table, R, o, lse, p_out);
+}
+
 int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                  int64_t Nk, int64_t d, float scale, int causal, double *o,
+                  int64_t Nk, int64_t d, double scale, int causal, double *o,
                   double *lse, double *p_out) {
     return attn_ref_fp64_window(q, k, v, key_lens, B, H, Nq, Nk, d, scale, causal, -1,
                                 o, lse, p_out);
@@ -211,7 +261,7 @@ int attn_ref_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  */
 int attn_ref_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const int32_t *key_lens, int64_t B, int64_t H, int64_t Nq,
-                       int64_t Nk, int64_t d, float scale, int causal,
+                       int64_t Nk, int64_t d, double scale, int causal,
                        const int64_t *row_ids, int64_t n, double *o_rows,
                        double *lse_rows) {
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0 || n < 0) return -1;
@@ -236,7 +286,8 @@ int attn_ref_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const int64_t b = bh / H;
                 const int64_t lim = row_limit(i, b, key_lens, Nq, Nk, causal);
                 one_row(q + r * d, k + bh * Nk * d, v + bh * Nk * d, Nk, d, sc,
-                        0, lim, 0.0, i + (Nk - Nq), s_row, p_row, o_rows + t * d, lse_rows + t);
+                        0, lim, 0.0, i + (Nk - Nq), NULL, 0, s_row, p_row, o_rows + t * d,
+                        lse_rows + t);
             }
         }
         free(s_row);

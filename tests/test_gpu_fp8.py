@@ -12,6 +12,13 @@ In units of e_j (divide by F >= 1): err_j <= max(2^-4 e_j, min(e_j, 2^-10)).  He
     |O'_c - O_c| <= sum_j err_j |V_jc - O_c| / (sum_j e_j - sum_j err_j),
 plus fp32 accumulation (n 2^-22 sum_j w_j |V_jc|, generous for tensor-core sums),
 the bf16 rounding of O (2^-8 |O_c|) and a 2 % slack for the exp2 approximations.
+The oracle's score factor is the exact product c = scale * q_descale * k_descale;
+the kernel applies c' = fp32(fp32(scale * q_descale) * k_descale), |c'/c - 1| <=
+2^-23 (two fp32 roundings).  That scales every score S_j by the same (1 + delta),
+which moves each weight e_j by a factor within exp(+-eta), eta = 2^-22 max_j |S_j|
+(|S_j - max S| <= 2 max |S|); the output then moves by at most
+eta / (1 - eta) * sum_j (e_j / E) |V_jc - O_c|, which is added to the bound (and
+the LSE by at most 2^-23 max |S|, far inside the LSE tolerance).
 The LSE comes from the unrounded fp32 sums: |dLSE| <= 1e-3 as for bf16 inputs.
 Fully masked rows: O = +0, LSE = -inf exactly.
 """
@@ -63,7 +70,8 @@ def _visible(Nq, Nk, causal, kl):
 
 def bound_rows(qf, kf, vf, s_eff, vis_rows, o_ref_rows):
     """Per-element bound of the derivation above for a set of rows of one (b, h).
-    qf [n, d], kf/vf [Nk, d] dequantised (vf includes v_descale); vis_rows [n, Nk]."""
+    qf [n, d], kf/vf [Nk, d] dequantised (vf includes v_descale); vis_rows [n, Nk];
+    s_eff the exact score factor scale * q_descale * k_descale (fp64)."""
     S = (qf @ kf.T) * s_eff
     S = np.where(vis_rows, S, -np.inf)
     mx = S.max(axis=1, keepdims=True)
@@ -73,12 +81,18 @@ def bound_rows(qf, kf, vf, s_eff, vis_rows, o_ref_rows):
     den = np.maximum(E - err.sum(axis=1, keepdims=True), 1e-300)
     n = vis_rows.sum(axis=1, keepdims=True)
     t_p = np.empty_like(o_ref_rows)
+    t_w = np.empty_like(o_ref_rows)
     for r0 in range(0, len(o_ref_rows), 16):                        # [16, Nk, d] at a time
         dev = np.abs(vf[None, :, :] - o_ref_rows[r0:r0 + 16, None, :])
         t_p[r0:r0 + 16] = np.einsum("rj,rjc->rc", err[r0:r0 + 16], dev)
+        t_w[r0:r0 + 16] = np.einsum("rj,rjc->rc", e[r0:r0 + 16], dev)
     t_p /= den
+    # the kernel's fp32 fold of the score factor (see the module docstring)
+    s_abs = np.where(vis_rows, np.abs(np.where(vis_rows, S, 0.0)), 0.0).max(axis=1, keepdims=True)
+    eta = 2.0 ** -22 * s_abs
+    t_fold = eta / (1.0 - eta) * t_w / np.maximum(E, 1e-300)
     t_acc = n * 2.0 ** -22 * (e @ np.abs(vf)) / np.maximum(E, 1e-300)
-    return 1.02 * (t_p + t_acc) + 2.0 ** -8 * np.abs(o_ref_rows) + 1e-6
+    return 1.02 * (t_p + t_acc) + t_fold + 2.0 ** -8 * np.abs(o_ref_rows) + 1e-6
 
 
 def check(o, lse, o_ref, lse_ref, bound, what):
@@ -121,7 +135,7 @@ def test_fp8_matches_oracle_within_the_derived_bound(case):
     kl_arr = None if kl is None else np.array(kl, np.int32)
     o, lse = run_fp8(q8, k8, v8, scale, qd, kd, vd, causal, kl_arr)
     o_ref, lse_ref = oracle.attn_ref_e4m3(q8, k8, v8, scale, qd, kd, vd, causal, kl_arr)
-    s_eff = np.float32(np.float64(scale) * qd * kd)
+    s_eff = np.float64(np.float32(scale)) * np.float64(np.float32(qd)) * np.float64(np.float32(kd))
     bound = np.zeros_like(o_ref)
     for b in range(B):
         vis = _visible(Nq, Nk, causal, Nk if kl is None else min(max(kl[b], 0), Nk))
@@ -167,7 +181,8 @@ def test_fp8_full_size_sampled_rows():
                                      [0, w.Nq - 1, w.Nq, w.B * w.H * w.Nq - 1]])).astype(np.int64)
     o_ref, lse_ref = oracle.attn_ref_rows_e4m3(x["q8"], x["k8"], x["v8"], w.scale, x["q_descale"],
                                                x["k_descale"], x["v_descale"], rows, w.causal)
-    s_eff = float(np.float32(np.float64(w.scale) * x["q_descale"] * x["k_descale"]))
+    s_eff = (np.float64(np.float32(w.scale)) * np.float64(np.float32(x["q_descale"]))
+             * np.float64(np.float32(x["k_descale"])))
     o_f = o.reshape(-1, w.d)[rows]
     l_f = lse.reshape(-1)[rows]
     bound = np.zeros_like(o_ref)

@@ -378,6 +378,95 @@ def test_bias_matches_torch_sdpa_with_an_additive_mask(causal, W):
     assert np.all(np.isneginf(lse[~has]))
 
 
+# ---------------------------------------------------------------- custom positional bias table
+# "FlashAttention：把注意力从公式写成数据流", section "精度、掩码和边界情况", lists
+# custom positional bias among the mask variants.  Reading: a per-head table of
+# 2R+1 values indexed by the key's position relative to the query's diagonal
+# position, clamped to [-R, R], added to the scaled scores.
+
+def _table(H, R, seed, sigma=1.0):
+    return (np.random.default_rng(seed).standard_normal((H, 2 * R + 1)) * sigma).astype(np.float32)
+
+
+def test_zero_table_is_no_bias():
+    q, k, v = _rand(2, 3, 9, 14, 8, 40)
+    kl = np.array([14, 6], np.int32)
+    for causal, W in ((False, -1), (True, -1), (True, 4)):
+        o0, l0 = oracle.attn_ref_window(q, k, v, 0.2, W, causal, kl)
+        o1, l1 = oracle.attn_ref_bias_table(q, k, v, 0.2, np.zeros((3, 7), np.float32), causal, kl, W)
+        assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_constant_table_shifts_only_the_lse():
+    # a constant bias c on every visible score: P and O unchanged, LSE + c
+    q, k, v = _rand(1, 2, 10, 12, 8, 41)
+    o0, l0 = oracle.attn_ref(q, k, v, 0.3, True)
+    c = np.float32(1.75)
+    o1, l1 = oracle.attn_ref_bias_table(q, k, v, 0.3, np.full((2, 9), c, np.float32), True)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l0 + float(c), rtol=0, atol=1e-13)
+
+
+def test_table_with_zero_query_is_its_softmax_weighting():
+    # q = 0: row i's scores are the table entries of its relative positions alone,
+    # so LSE_i = ln sum_j e^{T[clamp(j - i, -R, R) + R]} and O_i is the matching
+    # weighted mean of the visible value rows; R = 3 < N makes the clamp matter
+    B, H, N, d, R = 1, 2, 11, 8, 3
+    _, k, v = _rand(B, H, N, N, d, 42)
+    q = np.zeros((B, H, N, d), np.uint16)
+    tab = _table(H, R, 43)
+    o, lse = oracle.attn_ref_bias_table(q, k, v, 0.3, tab, False, None)
+    vf = bf16_bits_to_f32(v).astype(np.float64)
+    for h in range(H):
+        for i in range(N):
+            rel = [min(max(j - i, -R), R) for j in range(N)]
+            w = [math.exp(float(tab[h, r + R])) for r in rel]
+            assert abs(lse[0, h, i] - math.log(sum(w))) <= 1e-12
+            ref = sum(w[j] * vf[0, h, j] for j in range(N)) / sum(w)
+            np.testing.assert_allclose(o[0, h, i], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,W,R", [(True, -1, 40), (False, -1, 40), (True, 5, 40),
+                                        (False, -1, 4), (True, -1, 2)])
+def test_bias_table_matches_torch_sdpa_with_an_additive_mask(causal, W, R):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+    B, H, Nq, Nk, d = 2, 2, 11, 17, 8
+    q, k, v = _rand(B, H, Nq, Nk, d, 44)
+    kl = np.array([17, 9], np.int32)
+    tab = _table(H, R, 45 + R)
+    scale = 0.2
+    o, lse = oracle.attn_ref_bias_table(q, k, v, scale, tab, causal, kl, W)
+    tq, tk, tv = (torch.from_numpy(bf16_bits_to_f32(x).astype(np.float64)) for x in (q, k, v))
+    i = np.arange(Nq)[:, None] + (Nk - Nq)
+    j = np.arange(Nk)[None, :]
+    idx = np.clip(j - i, -R, R) + R
+    bias = np.zeros((B, H, Nq, Nk))
+    for b in range(B):
+        vis = j < kl[b]
+        if causal:
+            vis = vis & (j <= i)
+        if W >= 0:
+            vis = vis & (j >= i - W)
+        for h in range(H):
+            bias[b, h] = np.where(vis, tab[h][idx].astype(np.float64), -np.inf)
+    tb = torch.from_numpy(bias)
+    ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=tb,
+                                         scale=float(np.float32(scale))).numpy()
+    ref_lse = torch.logsumexp(torch.einsum("bhid,bhjd->bhij", tq, tk) * float(np.float32(scale))
+                              + tb, dim=-1).numpy()
+    has = np.isfinite(ref_lse)
+    np.testing.assert_allclose(o[has], ref[has], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[has], ref_lse[has], rtol=0, atol=1e-12)
+    assert np.all(np.isneginf(lse[~has]))
+
+
+def test_bias_table_rejects_an_even_width():
+    q, k, v = _rand(1, 2, 4, 4, 8, 46)
+    with pytest.raises(ValueError):
+        oracle.attn_ref_bias_table(q, k, v, 0.2, np.zeros((2, 6), np.float32))
+
+
 def test_varlen_of_equal_lengths_is_the_dense_problem():
     # packing B equal-length sequences token-major is a relayout of the dense batch
     B, H, N, d = 3, 2, 9, 8
@@ -468,6 +557,24 @@ def test_e4m3_zero_query_gives_the_scaled_mean_of_values():
         n = i + (Nk - Nq) + 1
         np.testing.assert_allclose(o[0, 0, i], 0.5 * vf[:n].mean(axis=0), rtol=0, atol=1e-12)
         assert abs(lse[0, 0, i] - math.log(n)) < 1e-13
+
+
+def test_e4m3_score_factor_is_the_exact_product():
+    # One visible key: LSE = scale * qd * kd * (q8 . k8) in closed form, with the
+    # product of the three fp32 factors taken exactly (the definition of the
+    # dequantised scores), not folded into one fp32 number first.
+    d = 8
+    q8 = np.array([[[[0x38, 0x40, 0x30, 0xB8, 0x3C, 0x28, 0x44, 0x34]]]], np.uint8)
+    k8 = np.array([[[[0x3A, 0xB0, 0x38, 0x2C, 0x40, 0x36, 0xB4, 0x38]]]], np.uint8)
+    v8 = np.full((1, 1, 1, d), 0x38, np.uint8)
+    scale, qd, kd = 0.1, 1.0 / 3.0, 0.7
+    f = lambda x: np.float64(np.float32(x))
+    dot = float(oracle.e4m3_to_f64(q8)[0, 0, 0] @ oracle.e4m3_to_f64(k8)[0, 0, 0])
+    exact = f(scale) * f(qd) * f(kd) * dot
+    folded = float(np.float32(np.float32(np.float32(scale) * np.float32(qd)) * np.float32(kd))) * dot
+    assert abs(folded - exact) > 1e-9 * abs(exact)     # the two readings differ here
+    _, lse = oracle.attn_ref_e4m3(q8, k8, v8, scale, qd, kd, 1.0)
+    assert abs(lse[0, 0, 0] - exact) <= 1e-15 * abs(exact)
 
 
 def test_e4m3_rows_entry_matches_full_evaluation():
