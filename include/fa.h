@@ -133,6 +133,32 @@ FA_API int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, flo
                 fa_stream_t stream);
 
 /*
+ * fa_fwd_bias_table -- fa_fwd with a custom positional bias: any per-head
+ * function of the key's position relative to the query, given as a table.
+ * Key j of query i gets, added to its scaled score,
+ *     table[h * (2R+1) + clamp(j - (i + N_k - N_q), -R, R) + R]
+ * (R = radius; relative positions beyond +-R use the table's end values), so
+ *   S_ij = scale * q_i . k_j + bias,  O and LSE as fa_fwd (the LSE includes
+ * the bias).  This is the general "custom positional bias" among the mask
+ * variants of "FlashAttention：把注意力从公式写成数据流", section
+ * "精度、掩码和边界情况"; a learned relative-position bias, or any distance
+ * penalty, is one table.
+ *
+ *   table         device fp32 [H, 2*radius+1], 4-byte aligned, non-NULL,
+ *                 natural-log units (the same units as scale * q . k); finite
+ *                 values (NaN/Inf propagate like NaN/Inf inputs).  Read only.
+ *   radius        R, 0 .. 2^30.
+ *   window_left   < 0: no window; >= 0: as fa_fwd_window.
+ *   other arguments, ownership and errors as fa_fwd; FA_ERR_INVALID_ARG for a
+ *   NULL table or a radius out of range, FA_ERR_MISALIGNED for an unaligned
+ *   table.
+ */
+FA_API int fa_fwd_bias_table(const void *q, const void *k, const void *v, void *o, float *lse,
+                             int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                             const int32_t *key_lens, const float *table, int radius,
+                             int window_left, fa_stream_t stream);
+
+/*
  * fa_fwd_fp8 -- fa_fwd on 8-bit E4M3 inputs with per-tensor scales: computes
  * the attention of the dequantised tensors Q = q_descale * Q8,
  * K = k_descale * K8, V = v_descale * V8, i.e.
@@ -149,10 +175,12 @@ FA_API int fa_fwd_bias(const void *q, const void *k, const void *v, void *o, flo
  *               0x7F/0xFF NaN), [B,H,N_q|N_k|N_k,d] contiguous, 16-byte aligned.
  *   o           device bf16 [B,H,N_q,d], 16-byte aligned.
  *   lse         device fp32 [B,H,N_q], 4-byte aligned.
- *   d           128 only (FA_ERR_UNSUPPORTED otherwise).
+ *   d           64 or 128 (FA_ERR_UNSUPPORTED otherwise).
  *   q_descale, k_descale, v_descale   finite, > 0 (FA_ERR_INVALID_ARG
- *               otherwise); scale * q_descale * k_descale is rounded once to
- *               fp32 and must stay finite and > 0.
+ *               otherwise).  The kernel applies the product
+ *               scale * q_descale * k_descale as one fp32 number (two fp32
+ *               roundings, a relative change of at most 2^-23 in every score);
+ *               it must stay finite and > 0.
  *   other arguments, ownership, empty cases and errors as fa_fwd.
  */
 FA_API int fa_fwd_fp8(const void *q8, const void *k8, const void *v8, void *o, float *lse,
@@ -265,10 +293,12 @@ FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *o, flo
  * Same operation, masks, layouts and outputs as fa_fwd.  The K/V tiles each
  * 128-row query block must visit are cut into num_splits contiguous ranges;
  * one CTA per (range, query block, head, batch) computes that range's
- * normalised partial output O_s and log-sum-exp LSE_s into the workspace, and
- * a second kernel merges them per row: with M = max_s LSE_s and
+ * normalised partial output O_s and log-sum-exp LSE_s into the workspace and
+ * counts its arrival for its query block; the last of the block's CTAs to
+ * arrive merges the ranges of the block's rows: with M = max_s LSE_s and
  * w_s = exp(LSE_s - M), O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s
- * (a row with no visible key in any range: O = 0, LSE = -inf).  This is the
+ * (a row with no visible key in any range: O = 0, LSE = -inf).  One memset of
+ * the arrival counters and one kernel launch per call.  This is the
  * decode / FlashDecoding case "FlashAttention：把注意力从公式写成数据流"
  * (section "端侧与专用加速器") and "[2205.14135] FlashAttention: Fast and
  * Memory-Efficient Exact Attention with IO-Awareness" point to, merged with the
@@ -278,18 +308,20 @@ FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *o, flo
 
 /*
  * fa_splitkv_num_splits -- a range count for this problem: 1 when the plain
- * grid (one CTA per 128 query rows and head) already covers 4/5 of B200's 148
- * SMs, else as many ranges as keep the grid within one wave (one CTA per SM),
- * with at least two K/V tiles (256 keys) per range and at most 256 ranges.
- * Returns 1 for empty or invalid sizes.  Pure host arithmetic.
+ * grid (one CTA per 128 query rows and head) already covers 4/5 of the current
+ * device's SMs, else as many ranges as keep the grid within one wave (one CTA
+ * per SM), with at least two K/V tiles (256 keys) per range and at most 256
+ * ranges.  The SM count is the current device's multiProcessorCount (148 on a
+ * B200); with no device visible it is taken as 148.  Returns 1 for empty or
+ * invalid sizes.  Host arithmetic plus that one device query.
  */
 FA_API int fa_splitkv_num_splits(int B, int H, int N_q, int N_k);
 
 /*
  * fa_fwd_splitkv_workspace_size -- bytes of device workspace fa_fwd_splitkv
- * needs: num_splits*B*H*N_q*d fp32 partial outputs followed by
- * num_splits*B*H*N_q fp32 partial LSEs, each 256-byte aligned.  Returns 0 for
- * invalid sizes or num_splits outside [1, 256].
+ * needs: num_splits*B*H*N_q*d fp32 partial outputs, num_splits*B*H*N_q fp32
+ * partial LSEs and ceil(N_q/128)*B*H int32 arrival counters, each part 256-byte
+ * aligned.  Returns 0 for invalid sizes or num_splits outside [1, 256].
  */
 FA_API size_t fa_fwd_splitkv_workspace_size(int B, int H, int N_q, int d, int num_splits);
 
@@ -359,6 +391,24 @@ FA_API int fa_get_device_status(fa_stream_t stream);
  * The CUDA context stays usable afterwards.
  */
 FA_API int fa_selftest_wait_timeout(unsigned long long limit_cycles, fa_stream_t stream);
+
+/*
+ * fa_selftest_fwd_timeout -- failure-detection self test of the forward
+ * kernel's own wind-down.  Runs the fa_fwd kernel (arguments as fa_fwd, no
+ * key_lens) with every pipeline wait bounded by `limit_cycles` SM clock cycles
+ * (1 .. 2^32) instead of the default of about a second, synchronises `stream`
+ * and returns what fa_get_device_status reports.  With a limit of a few
+ * cycles some wait runs out: that CTA and every role in it stop, each role
+ * first waiting (with the default limit) for the copies and MMAs it has
+ * already issued, so no asynchronous work lands in released shared memory or
+ * TMEM; the call returns FA_ERR_DEVICE_TIMEOUT and the CUDA context stays
+ * usable.  o and lse then hold unspecified values.  N_k must be > 0 and
+ * B*H*N_q > 0 (otherwise nothing would wait: FA_ERR_INVALID_ARG).
+ */
+FA_API int fa_selftest_fwd_timeout(const void *q, const void *k, const void *v, void *o,
+                                   float *lse, int B, int H, int N_q, int N_k, int d,
+                                   float scale, int causal, unsigned long long limit_cycles,
+                                   fa_stream_t stream);
 
 /*
  * fa_last_error -- the CUDA call and error text behind the most recent

@@ -61,6 +61,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                         vp, vp, i32, vp]
             lib.fa_fwd_bias.restype = i32
+            lib.fa_fwd_bias_table.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                              i32, vp, vp, i32, i32, vp]
+            lib.fa_fwd_bias_table.restype = i32
             lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32,
                                        f32, i32, vp, vp]
             lib.fa_fwd_fp8.restype = i32
@@ -93,6 +96,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_get_device_status.restype = i32
             lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
             lib.fa_selftest_wait_timeout.restype = i32
+            lib.fa_selftest_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                    f32, i32, ctypes.c_ulonglong, vp]
+            lib.fa_selftest_fwd_timeout.restype = i32
             lib.fa_last_error.argtypes = []
             lib.fa_last_error.restype = ctypes.c_char_p
             lib.fa_version.argtypes = []
@@ -167,6 +173,18 @@ def fa_fwd_bias(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, slo
                                     int(window_left), _stream(stream))
     if check and st != FA_OK:
         raise FaError(st, "fa_fwd_bias")
+    return st
+
+
+def fa_fwd_bias_table(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, key_lens, table, radius,
+                      window_left=-1, stream=None, check=True) -> int:
+    """``fa_fwd_bias_table`` of include/fa.h: forward with a custom positional bias table."""
+    st = load_library().fa_fwd_bias_table(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse),
+                                          int(B), int(H), int(N_q), int(N_k), int(d), float(scale),
+                                          int(bool(causal)), _addr(key_lens), _addr(table),
+                                          int(radius), int(window_left), _stream(stream))
+    if check and st != FA_OK:
+        raise FaError(st, "fa_fwd_bias_table")
     return st
 
 
@@ -268,6 +286,14 @@ def fa_get_device_status(stream=None) -> int:
 def fa_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:
     """``fa_selftest_wait_timeout`` of include/fa.h (bounded-wait self test)."""
     return int(load_library().fa_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
+
+
+def fa_selftest_fwd_timeout(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, limit_cycles,
+                            stream=None) -> int:
+    """``fa_selftest_fwd_timeout`` of include/fa.h: the forward kernel with a short wait limit."""
+    return int(load_library().fa_selftest_fwd_timeout(
+        _addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(H), int(N_q), int(N_k),
+        int(d), float(scale), int(bool(causal)), int(limit_cycles), _stream(stream)))
 
 
 def attention(q, k, v, causal=False, key_lens=None, scale=None, stream=None):

@@ -38,6 +38,9 @@ constexpr long long kHeadGroupL2Bytes = (long long)FA_HEAD_GROUP_MB << 20;
 // the plain order measured faster (GPT-2-sized causal problems, N = 1024)
 constexpr unsigned kHeadGroupMinBlocks = 32;
 constexpr int kMaxDevices = 64;
+// largest relative-position radius of a bias table (2^30: the table's
+// 2R+1 entries and every clamped index stay within int range)
+constexpr int kMaxBiasRadius = 1 << 30;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -100,6 +103,21 @@ int prepare_device(int dev) {
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128, true>::kSmemBytes);
         if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<64, true>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false, false, false, fa::kBiasSlopes>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, false, fa::kBiasSlopes>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false, false, false, fa::kBiasTable>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, false, fa::kBiasTable>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      fa::BwdCfg<64>::kSmemBytes);
         if (e == cudaSuccess)
@@ -140,27 +158,30 @@ int validate(const void* q, const void* k, const void* v, const void* o, const v
     return FA_OK;
 }
 
-// [B,H,N,d] viewed as a 4-D tensor (d, N, H, B), 128B swizzle, box of one 128-byte
-// row segment x 128 rows: 64 bf16 columns, or (e4m3 = true) 128 one-byte columns.
+// [B,H,N,d] viewed as a 4-D tensor (d, N, H, B), box of one swizzle span x 128
+// rows: 128B swizzle with 64 bf16 or 128 one-byte (e4m3) columns, or, for rows of
+// 64 one-byte elements, 64B swizzle with 64 columns (the kernel's Cfg geometry).
 bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, bool e4m3 = false) {
     EncodeTiledFn enc = encoder();
     if (enc == nullptr) return false;
     const cuuint64_t eb = e4m3 ? 1 : 2;
+    const cuuint64_t span = (cuuint64_t)d * eb < 128 ? (cuuint64_t)d * eb : 128;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)d * eb, (cuuint64_t)N * d * eb, (cuuint64_t)H * N * d * eb};
-    const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), (cuuint32_t)fa::kBlockM, 1, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)(span / eb), (cuuint32_t)fa::kBlockM, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               span == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Split-KV: partial results in the workspace, then the combine kernel.
+// Split-KV: partial results and per-block arrival counters in the workspace.
 struct SplitParts {
     int num_splits;   // 0: plain forward
     float* o_part;
     float* lse_part;
+    int* counter;     // [B, H, query blocks]
 };
 
 // Packed [T, H, d] bf16 viewed as (d, H, T, 1), box 64 x 1 x 128 x 1: the same
@@ -213,11 +234,19 @@ int launch_varlen(const void* q, const void* k, const void* v, void* o, float* l
     return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (packed variable-length)", e);
 }
 
+// Additive positional bias of a launch: none, per-head slopes, or a per-head table.
+struct BiasArgs {
+    int mode;             // fa::kBiasNone / kBiasSlopes / kBiasTable
+    const float* ptr;     // slopes [H] or table [H, 2*radius+1]
+    int radius;
+};
+
 // kF8: E4M3 Q, K, V (plain single-pass path only); o_scale multiplies O.
 template <int D, bool kF8 = false>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
-           float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr},
-           int window_left = -1, const float* slopes = nullptr, float o_scale = 1.f) {
+           float scale, int causal, const int32_t* key_lens, cudaStream_t stream, SplitParts sp = {0, nullptr, nullptr, nullptr},
+           int window_left = -1, BiasArgs bias = {fa::kBiasNone, nullptr, 0}, float o_scale = 1.f,
+           unsigned long long wait_limit = kWaitLimitCycles) {
     CUtensorMap tq, tk, tv, to;
     // With no keys the K/V maps are never read; give them a valid 1-row shape.
     const void* kp = N_k > 0 ? k : q;
@@ -239,11 +268,15 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.window_left = window_left;
-    p.slopes = slopes;
-    p.wait_limit = kWaitLimitCycles;
+    p.slopes = bias.mode == fa::kBiasSlopes ? bias.ptr : nullptr;
+    p.bias_table = bias.mode == fa::kBiasTable ? bias.ptr : nullptr;
+    p.bias_radius = bias.radius;
+    p.wait_limit = wait_limit;
     p.num_splits = sp.num_splits > 0 ? sp.num_splits : 1;
     p.o_part = sp.o_part;
     p.lse_part = sp.lse_part;
+    p.split_counter = sp.counter;
+    p.o_out = reinterpret_cast<__nv_bfloat16*>(o);
     p.o_scale = o_scale;
     const int rows_per_cta = fa::kBlockM;
     const unsigned num_m = (unsigned)((N_q + rows_per_cta - 1) / rows_per_cta);
@@ -264,35 +297,55 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     } else {
     if (sp.num_splits <= 0) {
         dim3 grid(num_m, (unsigned)H, (unsigned)B);
-        fa::fa_fwd_sm100_kernel<D, false><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        if (bias.mode == fa::kBiasSlopes)
+            fa::fa_fwd_sm100_kernel<D, false, false, false, fa::kBiasSlopes>
+                <<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        else if (bias.mode == fa::kBiasTable)
+            fa::fa_fwd_sm100_kernel<D, false, false, false, fa::kBiasTable>
+                <<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+        else
+            fa::fa_fwd_sm100_kernel<D, false><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv,
+                                                                                                       to, p);
         const cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
     }
+    // the arrival counters start at zero (the workspace has no required contents)
+    cudaError_t e = cudaMemsetAsync(sp.counter, 0, sizeof(int) * (size_t)num_m * H * B, stream);
+    if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync (split-KV counters)", e);
     dim3 grid(num_m * (unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
     fa::fa_fwd_sm100_kernel<D, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail("kernel launch (split-KV partials)", e);
-    const long long rows = (long long)B * H * N_q;
-    fa::fa_splitkv_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-        sp.o_part, sp.lse_part, reinterpret_cast<__nv_bfloat16*>(o), lse, rows, sp.num_splits);
     e = cudaGetLastError();
-    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV combine)", e);
+    return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV)", e);
     }
 }
 
 constexpr int kMaxSplits = 256;
-constexpr int kNumSms = 148;   // B200
+constexpr int kDefaultNumSms = 148;   // B200, when no device can be queried
 
-// Workspace of the split-KV forward: O partials, then LSE partials, 256-byte aligned.
+// Streaming multiprocessors of the current device (kDefaultNumSms without one).
+int current_num_sms() {
+    int ndev = 0, dev = -1, n = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0 || cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return kDefaultNumSms;
+    }
+    return n;
+}
+
+// Workspace of the split-KV forward: O partials, LSE partials, then one int32
+// arrival counter per (query block, head, batch), each 256-byte aligned.
 struct SplitLayout {
-    size_t o_part, lse_part, total;
+    size_t o_part, lse_part, counter, total;
 };
 SplitLayout split_layout(int B, int H, int N_q, int d, int num_splits) {
     const size_t rows = (size_t)num_splits * B * H * N_q;
+    const size_t blocks = (size_t)((N_q + fa::kBlockM - 1) / fa::kBlockM) * B * H;
     SplitLayout L{};
     L.o_part = 0;
     L.lse_part = (rows * d * 4 + 255) / 256 * 256;
-    L.total = L.lse_part + (rows * 4 + 255) / 256 * 256;
+    L.counter = L.lse_part + (rows * 4 + 255) / 256 * 256;
+    L.total = L.counter + (blocks * 4 + 255) / 256 * 256;
     return L;
 }
 
@@ -437,12 +490,13 @@ int fa_splitkv_num_splits(int B, int H, int N_q, int N_k) {
     if (B <= 0 || H <= 0 || N_q <= 0 || N_k <= 0) return 1;
     const long long ctas = (long long)((N_q + fa::kBlockM - 1) / fa::kBlockM) * B * H;
     const int tiles = (N_k + fa::kBlockN - 1) / fa::kBlockN;
-    // One CTA fits per SM.  Once the plain grid covers most of the 148 SMs the
+    // One CTA fits per SM.  Once the plain grid covers most of the SMs the
     // K/V stream already runs at HBM speed and splitting only adds the merge;
     // below that, split into as many ranges as still fit in one wave, with at
     // least two K/V tiles per range.
-    if (ctas >= kNumSms * 4 / 5) return 1;
-    long long s = kNumSms / ctas;
+    const int num_sms = current_num_sms();
+    if (ctas >= num_sms * 4 / 5) return 1;
+    long long s = num_sms / ctas;
     const long long cap = tiles / 2 > 1 ? tiles / 2 : 1;
     if (s > cap) s = cap;
     if (s > kMaxSplits) s = kMaxSplits;
@@ -479,7 +533,8 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
     if (st != FA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part)};
+    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part),
+                        reinterpret_cast<int*>(ws + L.counter)};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }
@@ -547,11 +602,13 @@ int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o,
     void* scratch = nullptr;
     st = scratch_address(dev, &scratch);
     if (st != FA_OK) return st;
-    // Every partial the merge reads is written first, so nothing in the
-    // scratch has to start at zero.
+    // Every partial the merge reads is written first, and the arrival counters
+    // are zeroed on the stream before the kernel, so nothing in the scratch has
+    // to start at zero.
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(scratch);
-    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part)};
+    const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part),
+                        reinterpret_cast<int*>(ws + L.counter)};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }
@@ -574,7 +631,7 @@ int fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* l
     st = prepare_device(dev);
     if (st != FA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const SplitParts none{0, nullptr, nullptr};
+    const SplitParts none{0, nullptr, nullptr, nullptr};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, window_left);
 }
@@ -585,7 +642,6 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* l
     bool empty = false;
     int st = validate(q8, k8, v8, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
     if (st != FA_OK) return st;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
     for (const float x : {q_descale, k_descale, v_descale})
         if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
     // the scores' three factors, folded into the one scale the kernel applies
@@ -603,9 +659,11 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* l
     st = prepare_device(dev);
     if (st != FA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const SplitParts none{0, nullptr, nullptr};
-    return launch<128, true>(q8, k8, v8, o, lse, B, H, N_q, N_k, c, causal, key_lens, s, none, -1, nullptr,
-                             v_descale);
+    const SplitParts none{0, nullptr, nullptr, nullptr};
+    const BiasArgs nob{fa::kBiasNone, nullptr, 0};
+    if (d == 64) return launch<64, true>(q8, k8, v8, o, lse, B, H, N_q, N_k, c, causal, key_lens, s, none, -1, nob,
+                                         v_descale);
+    return launch<128, true>(q8, k8, v8, o, lse, B, H, N_q, N_k, c, causal, key_lens, s, none, -1, nob, v_descale);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N_q, int d) {
@@ -667,10 +725,39 @@ int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse
     st = prepare_device(dev);
     if (st != FA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const SplitParts none{0, nullptr, nullptr};
+    const SplitParts none{0, nullptr, nullptr, nullptr};
     const int wl = window_left < 0 ? -1 : window_left;
-    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
-    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, slopes);
+    const BiasArgs bias{fa::kBiasSlopes, slopes, 0};
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, bias);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, bias);
+}
+
+int fa_fwd_bias_table(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q,
+                      int N_k, int d, float scale, int causal, const int32_t* key_lens, const float* table,
+                      int radius, int window_left, fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
+    if (st != FA_OK) return st;
+    if (radius < 0 || radius > kMaxBiasRadius) return FA_ERR_INVALID_ARG;
+    if (empty) return FA_OK;
+    if (table == nullptr) return FA_ERR_INVALID_ARG;
+    if (!aligned(table, 4)) return FA_ERR_MISALIGNED;
+    int dev = -1;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const SplitParts none{0, nullptr, nullptr, nullptr};
+    const int wl = window_left < 0 ? -1 : window_left;
+    const BiasArgs bias{fa::kBiasTable, table, radius};
+    if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, bias);
+    return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, none, wl, bias);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
@@ -787,6 +874,34 @@ int fa_selftest_wait_timeout(unsigned long long limit_cycles, fa_stream_t stream
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("self-test kernel launch", e);
+    return fa_get_device_status(stream);
+}
+
+int fa_selftest_fwd_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q,
+                            int N_k, int d, float scale, int causal, unsigned long long limit_cycles,
+                            fa_stream_t stream) {
+    bool empty = false;
+    int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, nullptr, &empty);
+    if (st != FA_OK) return st;
+    if (limit_cycles < 1 || limit_cycles > (1ull << 32)) return FA_ERR_INVALID_ARG;
+    if (empty || N_k == 0) return FA_ERR_INVALID_ARG;   // nothing would wait
+    int ndev = 0, dev = -1;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+    }
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    st = prepare_device(dev);
+    if (st != FA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const SplitParts none{0, nullptr, nullptr, nullptr};
+    const BiasArgs nob{fa::kBiasNone, nullptr, 0};
+    st = (d == 64) ? launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, nullptr, s, none, -1, nob, 1.f,
+                                limit_cycles)
+                   : launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, nullptr, s, none, -1, nob, 1.f,
+                                 limit_cycles);
+    if (st != FA_OK) return st;
     return fa_get_device_status(stream);
 }
 

@@ -77,6 +77,10 @@ constexpr uint32_t kRegsControl = 104;
 constexpr int kSwizzleBoxBytes = 128 * 128;  // one 64-column x 128-row bf16 box
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale only if max grows > 2^8
 constexpr int kStatusTimeout = -6;           // FA_ERR_DEVICE_TIMEOUT
+// additive score bias of the kernel instantiation
+constexpr int kBiasNone = 0;     // plain scores
+constexpr int kBiasSlopes = 1;   // -slope_h * |i + off - j|
+constexpr int kBiasTable = 2;    // a per-head table indexed by the clamped relative position
 // named barriers (epilogue only): 1..4 join the warps of a lane quadrant, 5 spans all softmax warps
 constexpr uint32_t kBarQuadBase = 1;
 constexpr uint32_t kBarSoftmaxAll = 5;
@@ -88,7 +92,11 @@ struct FwdParams {
     float scale_log2;           // scale * log2(e), > 0
     int causal;
     int window_left;            // sliding window: keys before i+off-window_left are masked; < 0: none
-    const float* slopes;        // [H] additive positional bias -slopes[h]*|i+off-j|, or nullptr
+    const float* slopes;        // [H] additive positional bias -slopes[h]*|i+off-j| (kBias == kBiasSlopes)
+    // custom positional bias (kBias == kBiasTable): fp32 [H, 2*bias_radius+1];
+    // key j of query i gets bias_table[h][clamp(j - (i+off), -R, R) + R]
+    const float* bias_table;
+    int bias_radius;
     // packed variable-length mode only: sequence b holds query tokens
     // cu_q[b] .. cu_q[b+1]-1 and key tokens cu_k[b] .. cu_k[b+1]-1; Nq / Nk
     // are then the token totals, Q/O are [Nq, H, D], K/V [Nk, H, D], LSE [Nq, H]
@@ -101,6 +109,10 @@ struct FwdParams {
     int num_splits;
     float* o_part;              // [num_splits, B, H, Nq, D] fp32, O of the range / its own l
     float* lse_part;            // [num_splits, B, H, Nq] fp32, LSE of the range (-inf if empty)
+    // arrivals per (query block, h, b), [B, H, num query blocks], zero at launch: the
+    // last CTA of a query block to finish merges its ranges into o_out / lse
+    int* split_counter;
+    __nv_bfloat16* o_out;       // final O [B,H,Nq,D] of the split-KV mode
     // dense single-pass mode: > 1 reorders the CTAs' work (see the kernel); 0 or 1 keeps
     // blockIdx = (query block, h, b)
     int head_group;
@@ -110,23 +122,28 @@ struct FwdParams {
 
 // kF8 = false: bf16 Q, K, V and P (kind::f16 MMAs).  kF8 = true: E4M3 Q, K, V
 // with per-tensor descales, P rounded to E4M3 (kind::f8f6f4 MMAs, K = 32 per
-// instruction); d = 128 only, so a row is one 128-byte swizzle row.
+// instruction).  Shared-memory tiles are 128-row boxes whose rows are one
+// swizzle span wide: 128 bytes (128B swizzle) whenever a Q/K/V row has at
+// least 128 bytes, else 64 bytes (64B swizzle: E4M3 at d = 64).
 template <int D, bool kF8 = false>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(!kF8 || D == 128, "E4M3 inputs: d = 128");
     static constexpr int kElemBytes = kF8 ? 1 : 2;
-    static constexpr int kBoxCols = 128 / kElemBytes;            // elements per 128-byte box row
-    static constexpr int kBoxes = D * kElemBytes / 128;          // boxes per Q / K / V row
-    static constexpr int kOBoxes = D / 64;                       // boxes per bf16 O row
-    static constexpr int kTileBytes = kBlockM * D * kElemBytes;  // one Q / K / V tile
+    static constexpr int kRowBytes = D * kElemBytes;             // one Q / K / V row
+    static constexpr int kSwz = kRowBytes < 128 ? kRowBytes : 128;   // swizzle span (bytes)
+    static constexpr uint32_t kSwzMode = kSwz == 128 ? 2u : 4u;  // descriptor layout: 128B / 64B swizzle
+    static constexpr int kBoxBytes = kBlockM * kSwz;             // one box: 128 rows x one span
+    static constexpr int kBoxCols = kSwz / kElemBytes;           // elements per box row
+    static constexpr int kBoxes = kRowBytes / kSwz;              // boxes per Q / K / V row
+    static constexpr int kOBoxes = D / 64;                       // 128B-swizzled boxes per bf16 O row
+    static constexpr int kTileBytes = kBlockM * kRowBytes;       // one Q / K / V tile
     static constexpr int kKPerMma = 32 / kElemBytes;             // K extent of one MMA (32 bytes)
-    static constexpr int kStagesK = (kTileBytes == 16384) ? 4 : 2;   // K ring slots
-    static constexpr int kStagesV = (kTileBytes == 16384) ? 4 : 2;   // V ring slots
+    static constexpr int kStagesK = (kTileBytes <= 16384) ? 4 : 2;   // K ring slots
+    static constexpr int kStagesV = (kTileBytes <= 16384) ? 4 : 2;   // V ring slots
     // A V slot holds the tile (kBoxes boxes) followed by one box of ones: the
     // PV product runs with N = D + 16 and its last 16 output columns
     // accumulate the row sums of the rounded P it multiplies.
-    static constexpr int kVSlotBytes = kTileBytes + kSwizzleBoxBytes;
+    static constexpr int kVSlotBytes = kTileBytes + kBoxBytes;
     static constexpr uint32_t kOnesWord = kF8 ? 0x38383838u : 0x3F803F80u;   // 1.0 in E4M3 / bf16
     static constexpr int kNPV = D + 16;
     static constexpr int kStages = kStagesK + kStagesV;
@@ -151,10 +168,13 @@ struct Cfg {
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
     static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row]
     static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, lu [2][row] each
-    static constexpr int kSmemBytes = kEpiOff + 2 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
+    static constexpr int kSmemUsed = kEpiOff + 2 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
+    // One CTA per SM either way (it holds all 512 TMEM columns), so the smaller
+    // E4M3 layouts reserve as much shared memory as the bf16 d = 64 one.
+    static constexpr int kSmemBytes = kSmemUsed < 200 * 1024 ? 200 * 1024 : kSmemUsed;
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
     // The bf16 O tile is staged for its TMA store from the start of the Q
-    // buffer on; with 8-bit inputs it also covers the first K slot (idle by then).
+    // buffer on; with 8-bit inputs it also covers the first K slot(s) (idle by then).
     static_assert(kOBoxes * kSwizzleBoxBytes <= kVOff, "O staging area");
     // TMEM columns: the S buffer at 0..127, the P buffers (kPCols each: bf16
     // pairs or E4M3 quads) after it, then O (D columns) and its row-sum
@@ -178,15 +198,19 @@ struct Cfg {
                                          ((uint32_t)(kBlockM >> 4) << 24);
 };
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor with sm_100 version bits; `mode` is the
+// layout field: 2 = 128-byte swizzle, 4 = 64-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t mode) {
     uint64_t d = 0;
     d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;   // descriptor version for tcgen05
-    d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+    d |= (uint64_t)(mode & 7u) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return smem_desc(addr, lbo, sbo, 2u);
 }
 
 __device__ int g_fa_status;
@@ -205,6 +229,24 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
         if (*abort_flag) return false;
         if ((unsigned long long)(clock64() - t0) > limit) {
             *abort_flag = 1;
+            atomicExch(&g_fa_status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+// Bounded wait for this thread's own asynchronous work (a TMA copy it issued, or
+// the commit of its MMAs) when winding down: unlike wait_bounded it does not
+// give up when another role of the CTA has raised the abort flag, because
+// shared memory and TMEM must not be released while that work may still land.
+// The limit is the default one (about a second), not a caller's shorter limit.
+constexpr unsigned long long kDrainWaitLimit = 1ull << 31;
+__device__ __forceinline__ bool wait_own_work(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((unsigned long long)(clock64() - t0) > kDrainWaitLimit) {
             atomicExch(&g_fa_status, kStatusTimeout);
             return false;
         }
@@ -296,17 +338,81 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
     return c < kl ? (int)c : kl;
 }
 
-// kSplit = false: the whole forward (O and LSE).  kSplit = true: the first half
-// of the split-KV forward ("FlashAttention：把注意力从公式写成数据流", section
-// "端侧与专用加速器", and "[2205.14135] FlashAttention: Fast and
-// Memory-Efficient Exact Attention with IO-Awareness", its note on the decode
-// case): partial (O, LSE) for one contiguous range of K/V tiles, merged by
-// fa_splitkv_combine_kernel.
+// Split-KV merge, run by the 256 softmax threads of a CTA once its partial
+// (O_s, LSE_s) is in global memory: the CTA counts its arrival for its query
+// block, and the last of the block's num_splits CTAs to arrive merges every
+// range of the block's rows.  With M = max_s LSE_s and w_s = e^(LSE_s - M):
+//   O = sum_s w_s O_s / sum_s w_s,   LSE = M + ln sum_s w_s
+// (each O_s is normalised by its own range's sum, so w_s carries that sum;
+// this is the online softmax's running-max rule applied to whole ranges).  A
+// row whose ranges are all empty (M = -inf) gets O = 0, LSE = -inf; an empty
+// range has LSE_s = -inf, so w_s = 0 and its O_s (zeros) adds nothing.  Work
+// items are (row, 4 columns), spread over the 256 threads, so a decode block
+// with one row still loads its ranges' partials in parallel.  The counters are
+// zeroed on the stream before every launch.
+template <int D>
+__device__ __forceinline__ void split_merge(const FwdParams& p, uint8_t* flag_smem, int n_split, int num_m, int m_blk,
+                                            int m0, int h, int b) {
+    volatile int* const flag = reinterpret_cast<volatile int*>(flag_smem);
+    const size_t grp = ((size_t)b * p.H + h) * (size_t)num_m + (size_t)m_blk;
+    if (threadIdx.x == 0) {
+        // every softmax thread fenced its own partial stores before the barrier
+        // that preceded this arrival
+        const int old = atomicAdd(p.split_counter + grp, 1);
+        *flag = (old == n_split - 1) ? 1 : 0;
+    }
+    named_bar_sync(kBarSoftmaxAll, kSoftmaxWarps * 32);
+    if (!*flag) return;
+    __threadfence();   // the other ranges' partials, published before their arrivals
+    constexpr int kC4 = D / 4;
+    const int rows = min(kBlockM, p.Nq - m0);
+    const size_t rows_total = (size_t)p.B * p.H * (size_t)p.Nq;
+    const size_t row0 = ((size_t)b * p.H + h) * (size_t)p.Nq + (size_t)m0;
+    for (int it = threadIdx.x; it < rows * kC4; it += kSoftmaxWarps * 32) {
+        const int rr = it / kC4, c4 = it - rr * kC4;
+        const size_t rg = row0 + (size_t)rr;
+        float mx = -INFINITY;
+#pragma unroll 4
+        for (int sp = 0; sp < n_split; ++sp) mx = fmaxf(mx, __ldcg(p.lse_part + sp * rows_total + rg));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        if (mx != -INFINITY) {
+#pragma unroll 4
+            for (int sp = 0; sp < n_split; ++sp) {
+                const float ls = __ldcg(p.lse_part + sp * rows_total + rg);
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(p.o_part + (sp * rows_total + rg) * D) + c4);
+                const float w = (ls == -INFINITY) ? 0.f : expf(ls - mx);
+                acc.x = fmaf(w, v.x, acc.x);
+                acc.y = fmaf(w, v.y, acc.y);
+                acc.z = fmaf(w, v.z, acc.z);
+                acc.w = fmaf(w, v.w, acc.w);
+                wsum += w;
+            }
+        }
+        const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(p.o_out + rg * D + 4 * c4) = pk;
+        if (c4 == 0) p.lse[rg] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+    }
+}
+
+// kSplit = false: the whole forward (O and LSE).  kSplit = true: the split-KV
+// forward ("FlashAttention：把注意力从公式写成数据流", section "端侧与专用加速器",
+// and "[2205.14135] FlashAttention: Fast and Memory-Efficient Exact Attention
+// with IO-Awareness", its note on the decode case): partial (O, LSE) for one
+// contiguous range of K/V tiles, merged by the block's last CTA (split_merge).
 // kVarlen = true: packed variable-length batches (FwdParams::cu_q / cu_k);
 // the TMA maps then view [tokens, H, D] as (D, H, tokens, 1).
 // kF8 = true: E4M3 inputs (see Cfg); O is still bf16 and FwdParams::o_scale
 // (the V descale) multiplies it in the epilogue.
-template <int D, bool kSplit = false, bool kVarlen = false, bool kF8 = false>
+// kBias: kBiasNone, or an additive positional bias on the scores
+// ("FlashAttention：把注意力从公式写成数据流", section "精度、掩码和边界情况":
+// positional biases are among the mask variants): kBiasSlopes, a linear
+// distance penalty per head, or kBiasTable, any per-head function of the
+// relative position j - (i + off) given as a table, clamped at +-R.
+template <int D, bool kSplit = false, bool kVarlen = false, bool kF8 = false, int kBias = kBiasNone>
 __global__ void __launch_bounds__(kNumThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -442,9 +548,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tc_fence_before();
     }
     // the ones box of every V slot (TMA writes only the boxes before it)
-    for (int i = threadIdx.x; i < C::kStagesV * (kSwizzleBoxBytes / 16); i += kNumThreads) {
-        const int sl = i / (kSwizzleBoxBytes / 16);
-        const uint32_t a = ring_slot(1, sl) + (uint32_t)C::kTileBytes + (uint32_t)(i % (kSwizzleBoxBytes / 16)) * 16u;
+    for (int i = threadIdx.x; i < C::kStagesV * (C::kBoxBytes / 16); i += kNumThreads) {
+        const int sl = i / (C::kBoxBytes / 16);
+        const uint32_t a = ring_slot(1, sl) + (uint32_t)C::kTileBytes + (uint32_t)(i % (C::kBoxBytes / 16)) * 16u;
         asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(C::kOnesWord) : "memory");
     }
     fence_proxy_async_smem();   // visible to the tensor core's reads
@@ -468,7 +574,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 int qc1, qc2, qc3;
                 tile_coords(q_base, m0, qc1, qc2, qc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(q_tile + bx * kSwizzleBoxBytes, &tm_q, bar_q_full, bx * C::kBoxCols, qc1, qc2, qc3,
+                    tma_load_4d(q_tile + bx * C::kBoxBytes, &tm_q, bar_q_full, bx * C::kBoxCols, qc1, qc2, qc3,
                                 policy_evict_first());
             }
             bool ok = true;
@@ -482,15 +588,17 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 int kc1, kc2, kc3;
                 tile_coords(k_base, (t0 + j) * kBlockN, kc1, kc2, kc3);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(ring_slot(rg, s) + bx * kSwizzleBoxBytes, tm, bar_full(rg, s), bx * C::kBoxCols, kc1, kc2,
+                    tma_load_4d(ring_slot(rg, s) + bx * C::kBoxBytes, tm, bar_full(rg, s), bx * C::kBoxCols, kc1, kc2,
                                 kc3, pol_kv);
             }
-            if (!ok) {
-                // wind down: let every copy still in flight (at most one per
-                // slot, the newest ones) land before the CTA exits
-                for (int c2 = (j > ns ? j - ns : 0); c2 < j; ++c2)
-                    (void)wait_bounded(bar_full(rg, c2 % ns), (uint32_t)((c2 / ns) & 1), abort_flag, p.wait_limit);
-            }
+            // Before the CTA can exit, every copy this producer issued that may
+            // still be in flight (Q, and at most one per slot, the newest ones)
+            // must have landed.  On the normal path the consumers have waited for
+            // them already (or are about to); after a timeout anywhere in the CTA
+            // they may not have, so this wait ignores the abort flag.
+            if (rg == 0) (void)wait_own_work(bar_q_full, 0);
+            for (int c2 = (j > ns ? j - ns : 0); c2 < j; ++c2)
+                (void)wait_own_work(bar_full(rg, c2 % ns), (uint32_t)((c2 / ns) & 1));
         }
         __syncwarp();
     } else {
@@ -513,10 +621,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     const uint32_t slot = ring_slot(0, sl);
 #pragma unroll
                     for (int kk = 0; kk < D * C::kElemBytes / 32; ++kk) {
-                        // 32 bytes of every row per MMA: 4 steps per 128-byte box
-                        const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
-                        const uint64_t a = smem_desc_sw128(q_tile + koff, 16, 1024);
-                        const uint64_t bb = smem_desc_sw128(slot + koff, 16, 1024);
+                        // 32 bytes of every row per MMA, kSwz / 32 steps per box
+                        const uint32_t koff =
+                            (uint32_t)((kk * 32 / C::kSwz) * C::kBoxBytes + (kk * 32) % C::kSwz);
+                        const uint64_t a = smem_desc(q_tile + koff, 16, 8 * C::kSwz, C::kSwzMode);
+                        const uint64_t bb = smem_desc(slot + koff, 16, 8 * C::kSwz, C::kSwzMode);
                         if constexpr (kF8)
                             umma_ss_f8(tmem + C::col_s(i % C::kSBufs), a, bb, C::kIdescQK, kk > 0 ? 1u : 0u);
                         else
@@ -539,10 +648,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBlockN / C::kKPerMma; ++kk) {
                         // keys kK*kk .. kK*kk+kK-1 of P (kK = 16 bf16 or 32 E4M3): 8 TMEM
-                        // columns of P, kK 128-byte rows of the V slot per step
+                        // columns of P, kK rows (one swizzle span each) of the V slot per step
                         const uint32_t a_col = C::col_p(pb) + (uint32_t)(kk * 8);
                         const uint64_t bb =
-                            smem_desc_sw128(slot + (uint32_t)(kk * C::kKPerMma * 128), kSwizzleBoxBytes, 1024);
+                            smem_desc(slot + (uint32_t)(kk * C::kKPerMma * C::kSwz), C::kBoxBytes, 8 * C::kSwz,
+                                      C::kSwzMode);
                         if constexpr (kF8)
                             umma_ts_f8(tmem + C::kColO, tmem + a_col, bb, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                         else
@@ -553,9 +663,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
             }
             // drain: every MMA and commit of this CTA has landed before TMEM is
-            // freed (the barrier completes once both issuers have committed)
+            // freed (the barrier completes once both issuers have committed);
+            // this wait ignores the abort flag, so a wound-down CTA drains too
             umma_commit(bar_drain);
-            (void)wait_bounded(bar_drain, 0, abort_flag, p.wait_limit);
+            (void)wait_own_work(bar_drain, 0);
         }
         __syncwarp();
       }
@@ -570,8 +681,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int lim = row_key_limit(row, kl, off, p.causal);
         const int lo = row_key_start(row, off, p.window_left);   // 0 without a window
         // additive positional bias, in log2 units per unit of distance (warp-uniform switch)
-        const bool has_bias = p.slopes != nullptr;
-        const float alpha = has_bias ? p.slopes[h] * 1.4426950408889634f : 0.f;
+        constexpr bool has_bias = kBias != kBiasNone;
+        const float alpha = (kBias == kBiasSlopes) ? p.slopes[h] * 1.4426950408889634f : 0.f;
+        const float* const trow =
+            (kBias == kBiasTable) ? p.bias_table + (size_t)h * (2 * (size_t)p.bias_radius + 1) + p.bias_radius : nullptr;
         const float c = p.scale_log2;
         float m_seen = -INFINITY;  // newest reference max this thread knows (log2 units)
         float lu = 0.f;            // the same sum before rounding (for the LSE)
@@ -606,12 +719,27 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const int kbase = (t0 + j) * kBlockN;
             // warp-uniform: the element mask runs only on tiles that cross a row's key limit
             const bool masked = __any_sync(0xffffffffu, kbase + kBlockN > lim || kbase < lo);
-            if (has_bias) {
+            if constexpr (kBias == kBiasSlopes) {
                 // t_i = s_i * c - alpha * |row + off - (kbase + i)|; from here on the
                 // scores are in log2 units already (scale factor 1)
                 const float d0 = (float)(row + off - kbase);
 #pragma unroll
                 for (int i = 0; i < kBlockN; ++i) s[i] = fmaf(s[i], c, -alpha * fabsf(d0 - (float)i));
+            } else if constexpr (kBias == kBiasTable) {
+                // t_i = s_i * c + log2(e) * table[clamp(r0 + i, -R, R)], r0 the relative
+                // position of the tile's first key; tiles inside [-R, R] for the whole
+                // warp skip the clamp.  Masked keys are overwritten with -inf below.
+                const int R = p.bias_radius;
+                const int r0 = kbase - (row + off);
+                if (__all_sync(0xffffffffu, r0 >= -R && r0 + kBlockN - 1 <= R)) {
+#pragma unroll
+                    for (int i = 0; i < kBlockN; ++i)
+                        s[i] = fmaf(__ldg(trow + r0 + i), 1.4426950408889634f, s[i] * c);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kBlockN; ++i)
+                        s[i] = fmaf(__ldg(trow + min(max(r0 + i, -R), R)), 1.4426950408889634f, s[i] * c);
+                }
             }
             const float cs = has_bias ? 1.f : c;
             if (masked) {
@@ -807,8 +935,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 else
                     p.lse[((size_t)b * p.H + h) * (size_t)p.Nq + row] = lse;
             }
+        } else if constexpr (kSplit) {
+            // a wait ran out (the device status records it): leave an empty
+            // range (O = 0, LSE = -inf) rather than whatever the workspace held,
+            // so the merge adds nothing stale from an earlier call
+            if (row < p.Nq) {
+                float4* dst = reinterpret_cast<float4*>(
+                    p.o_part + ((((size_t)split * p.B + b) * p.H + h) * (size_t)p.Nq + row) * D + g * (D / 2));
+#pragma unroll
+                for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (g == 0) p.lse_part[(((size_t)split * p.B + b) * p.H + h) * (size_t)p.Nq + row] = -INFINITY;
+            }
         }
         fence_proxy_async_smem();
+        if constexpr (kSplit) __threadfence();   // this CTA's partials, before its arrival below
         const bool any_bad = named_bar_or(kBarSoftmaxAll, kSoftmaxWarps * 32, !good);
         if (!kSplit && !kVarlen && !any_bad && threadIdx.x == 0) {
             for (int bx = 0; bx < C::kOBoxes; ++bx)
@@ -816,6 +956,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             bulk_commit_group();
             bulk_wait_group_read0();
         }
+        if constexpr (kSplit) split_merge<D>(p, base_ptr + C::kMiscOff + 8, n_split, num_m, m_blk, m0, h, b);
         tc_fence_before();
     }
 
@@ -826,69 +967,5 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
 }
 
-// Second half of the split-KV forward: merge the partial results of the
-// K/V ranges of every query row.  With M = max_s LSE_s and w_s = e^(LSE_s - M):
-//   O = sum_s w_s O_s / sum_s w_s,   LSE = M + ln sum_s w_s
-// (each O_s is normalised by its own range's sum, so w_s carries that sum).
-// A row whose ranges are all empty (M = -inf) gets O = 0, LSE = -inf; an empty
-// range has LSE_s = -inf, so w_s = 0 and its O_s (zeros) adds nothing.
-// One warp per row; lane s holds the weights of ranges s, s+32, ...; each lane
-// owns D/32 consecutive output columns.
-template <int D>
-__global__ void __launch_bounds__(256)
-    fa_splitkv_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                              __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long rows, int n_split) {
-    constexpr int kCols = D / 32;
-    constexpr int kMaxPerLane = 8;   // n_split <= 256
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    float ls[kMaxPerLane];
-    float m = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < kMaxPerLane; ++t) {
-        const int sp = lane + 32 * t;
-        ls[t] = (sp < n_split) ? lse_part[(size_t)sp * rows + row] : -INFINITY;
-        m = fmaxf(m, ls[t]);
-    }
-#pragma unroll
-    for (int sh = 16; sh > 0; sh >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sh));
-    float wl[kMaxPerLane];
-    float wsum = 0.f;
-#pragma unroll
-    for (int t = 0; t < kMaxPerLane; ++t) {
-        wl[t] = (m == -INFINITY || ls[t] == -INFINITY) ? 0.f : expf(ls[t] - m);
-        wsum += wl[t];
-    }
-#pragma unroll
-    for (int sh = 16; sh > 0; sh >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, sh);
-    float acc[kCols];
-#pragma unroll
-    for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-    const float* src = o_part + (size_t)row * D + lane * kCols;
-    const size_t split_stride = (size_t)rows * D;
-#pragma unroll
-    for (int t = 0; t < kMaxPerLane; ++t) {
-        if (32 * t >= n_split) break;
-#pragma unroll 4
-        for (int k2 = 0; k2 < 32; ++k2) {
-            const int sp = 32 * t + k2;
-            if (sp >= n_split) break;
-            const float w = __shfl_sync(0xffffffffu, wl[t], k2);
-            const float* p2 = src + (size_t)sp * split_stride;
-#pragma unroll
-            for (int i = 0; i < kCols; i += 2) {
-                const float2 v = *reinterpret_cast<const float2*>(p2 + i);
-                acc[i] = fmaf(w, v.x, acc[i]);
-                acc[i + 1] = fmaf(w, v.y, acc[i + 1]);
-            }
-        }
-    }
-    const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(o + row * D + lane * kCols);
-#pragma unroll
-    for (int i = 0; i < kCols; i += 2) dst[i / 2] = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
-    if (lane == 0) lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
-}
 
 }  // namespace fa

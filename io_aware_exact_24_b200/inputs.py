@@ -30,6 +30,7 @@ import numpy as np
 
 TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_KEYLEN = 0, 1, 2, 3
 TENSOR_DO = 4   # upstream gradient dL/dO for the backward pass
+TENSOR_BIAS_TABLE = 5   # custom positional bias table
 
 
 @dataclasses.dataclass(frozen=True)
@@ -49,6 +50,7 @@ class Workload:
     seed: int = 0
     window_left: int = -1                          # sliding window (fa_fwd_window); -1 = none
     alibi: bool = False                            # additive positional bias with alibi_slopes(H)
+    bias_table_radius: int = -1                    # custom bias table of 2R+1 entries per head; -1 = none
 
     @property
     def flop(self) -> float:
@@ -183,6 +185,13 @@ def alibi_slopes(H: int) -> np.ndarray:
     return (2.0 ** (-8.0 * (np.arange(H) + 1) / H)).astype(np.float32)
 
 
+def bias_table(H: int, R: int, seed: int) -> np.ndarray:
+    """A custom positional bias table for fa_fwd_bias_table: fp32 [H, 2R+1] of
+    N(0, 1) samples (stream seed*16 + 5), one value per head and clamped relative
+    position."""
+    return _rng(seed, TENSOR_BIAS_TABLE).standard_normal(size=(H, 2 * R + 1), dtype=np.float32)
+
+
 # Mask variants: sliding-window (local) causal attention for fa_fwd_window, each
 # query seeing the 2048 keys before its position and itself; and the
 # causal_8000_d128 shape with the additive positional bias (fa_fwd_bias).
@@ -193,4 +202,9 @@ WINDOW_WORKLOADS = {
     "alibi_causal_8000_d128": Workload("alibi_causal_8000_d128", 2, 32, 8000, 8000, 128, True,
                                        float(np.float32(1 / math.sqrt(128))), 0.5, None, 5,
                                        alibi=True),
+    # the same shape with a custom positional bias table of 2*1024+1 entries per head
+    # (relative positions beyond +-1024 clamped)
+    "table_causal_8000_d128": Workload("table_causal_8000_d128", 2, 32, 8000, 8000, 128, True,
+                                       float(np.float32(1 / math.sqrt(128))), 0.5, None, 5,
+                                       bias_table_radius=1024),
 }

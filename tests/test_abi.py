@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("fa_fwd", "fa_fwd_host", "fa_fwd_host_workspace_size", "fa_status_string",
-                 "fa_get_device_status", "fa_version", "fa_selftest_wait_timeout"):
+                 "fa_get_device_status", "fa_version", "fa_selftest_wait_timeout",
+                 "fa_selftest_fwd_timeout"):
         assert must in names
 
 
@@ -132,7 +133,8 @@ def test_splitkv_workspace_size_formula(lib):
         rows = S * B * H * Nq
         need = binding.fa_fwd_splitkv_workspace_size(B, H, Nq, d, S)
         o_bytes = -(-rows * d * 4 // 256) * 256
-        assert need == o_bytes + -(-rows * 4 // 256) * 256
+        blocks = -(-Nq // 128) * B * H          # one int32 arrival counter per query block
+        assert need == o_bytes + -(-rows * 4 // 256) * 256 + -(-blocks * 4 // 256) * 256
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 96, 2) == 0
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 0) == 0
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 257) == 0
@@ -242,6 +244,49 @@ def test_bias_without_a_gpu_reports_no_device(lib):
     assert bias_call() == binding.FA_ERR_NO_DEVICE
 
 
+# ---------------------------------------------------------------- bias table entry point
+
+def table_call(table=P, radius=4, window_left=-1, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, Nq=8, Nk=8, d=64, scale=0.125, causal=1,
+             key_lens=None)
+    a.update(kw)
+    return binding.fa_fwd_bias_table(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                                     a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                                     a["key_lens"], table, radius, window_left, stream=0,
+                                     check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(table=None), binding.FA_ERR_INVALID_ARG),
+    (dict(table=P + 2), binding.FA_ERR_MISALIGNED),
+    (dict(radius=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(radius=(1 << 30) + 1), binding.FA_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0, table=None), binding.FA_OK),
+])
+def test_bias_table_argument_errors_before_any_cuda_call(lib, kw, code):
+    assert table_call(**kw) == code
+
+
+def test_bias_table_without_a_gpu_reports_no_device(lib):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert table_call() == binding.FA_ERR_NO_DEVICE
+    assert table_call(radius=0) == binding.FA_ERR_NO_DEVICE
+
+
+def test_selftest_fwd_timeout_argument_errors(lib):
+    f = lambda **kw: binding.fa_selftest_fwd_timeout(
+        P, P, P, P, P, kw.get("B", 1), 2, kw.get("Nq", 8), kw.get("Nk", 8), 64, 0.125, 1,
+        kw.get("limit", 2), stream=0)
+    assert f(limit=0) == binding.FA_ERR_INVALID_ARG
+    assert f(limit=(1 << 32) + 1) == binding.FA_ERR_INVALID_ARG
+    assert f(Nk=0) == binding.FA_ERR_INVALID_ARG
+    assert f(B=0) == binding.FA_ERR_INVALID_ARG
+
+
 # ---------------------------------------------------------------- packed variable-length entry point
 
 def varlen_call(**kw):
@@ -290,8 +335,8 @@ def fp8_call(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(d=64), binding.FA_ERR_UNSUPPORTED),
     (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
     (dict(qd=0.0), binding.FA_ERR_INVALID_ARG),
     (dict(kd=-1.0), binding.FA_ERR_INVALID_ARG),
     (dict(vd=float("nan")), binding.FA_ERR_INVALID_ARG),
@@ -303,7 +348,8 @@ def fp8_call(**kw):
     (dict(v=P + 4), binding.FA_ERR_MISALIGNED),
     (dict(o=None), binding.FA_ERR_INVALID_ARG),
     (dict(B=0), binding.FA_OK),
-    (dict(Nq=0, d=64), binding.FA_ERR_UNSUPPORTED),
+    (dict(Nq=0, d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(Nq=0, d=64), binding.FA_OK),
 ])
 def test_fp8_argument_errors_before_any_cuda_call(lib, kw, code):
     assert fp8_call(**kw) == code
@@ -314,6 +360,7 @@ def test_fp8_without_a_gpu_reports_no_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert fp8_call() == binding.FA_ERR_NO_DEVICE
+    assert fp8_call(d=64) == binding.FA_ERR_NO_DEVICE
 
 
 # ---------------------------------------------------------------- backward entry point

@@ -24,8 +24,9 @@ from test_bwd_protocol_model import Barrier
 
 
 class Fwd:
-    def __init__(self, n, ns_k, ns_v, seed, p_rescale=0.3, slow=1.0, v_lat=(200, 3000)):
+    def __init__(self, n, ns_k, ns_v, seed, p_rescale=0.3, slow=1.0, v_lat=(200, 3000), n_s=1, n_p=3):
         self.rng = random.Random(seed)
+        self.n_s, self.n_p = n_s, n_p    # TMEM score buffers, P buffers
         self.v_lat = v_lat
         self.n, self.nsk, self.nsv, self.p_rescale, self.slow = n, ns_k, ns_v, p_rescale, slow
         self.now, self.seq, self.events, self.tc_free = 0.0, 0, [], 0.0
@@ -36,14 +37,15 @@ class Fwd:
         self.vf = [b(f"v_full{s}", 1) for s in range(ns_v)]
         self.ve = [b(f"v_empty{s}", 1) for s in range(ns_v)]
         self.s_full = [b(f"s_full{g}", 1) for g in range(2)]
-        self.s_free = b("s_free", 4)
-        self.p_full = [b(f"p_full{i}", 4) for i in range(3)]
-        self.pv_done = [b(f"pv_done{i}", 1) for i in range(3)]
+        self.s_free = [b(f"s_free{i}", 4) for i in range(n_s)]
+        self.p_full = [b(f"p_full{i}", 4) for i in range(n_p)]
+        self.pv_done = [b(f"pv_done{i}", 1) for i in range(n_p)]
         self.m_ready = [[b(f"m_ready{q}{g}", 1) for g in range(2)] for q in range(4)]
         self.drain = b("drain", 2)
         self.kslot, self.vslot = [None] * ns_k, [None] * ns_v
-        self.s_buf, self.s_reads = None, 0
-        self.p_buf = [None] * 3          # (tile, quadrants written)
+        self.s_buf = [None] * n_s        # tile held by each score buffer
+        self.s_reads = [0] * n_s         # quadrants that have read it
+        self.p_buf = [None] * n_p        # (tile, quadrants written)
         self.pv_done_count = 0           # PVs finished
         self.pv_started = -1             # last PV started
         self.mref = {}                   # (q, g) -> tile whose max it holds
@@ -140,21 +142,22 @@ def qk_issuer(m):
         return
     yield wait(m.q_full, 0)
     for i in range(m.n):
-        if i >= 1:
-            yield wait(m.s_free, i - 1)
+        sb = i % m.n_s
+        if i >= m.n_s:
+            yield wait(m.s_free[sb], (i - m.n_s) // m.n_s)
         s = i % m.nsk
         yield wait(m.kf[s], i // m.nsk)
 
-        def start(i=i, s=s):
+        def start(i=i, s=s, sb=sb):
             if m.kslot[s] != i:
                 m.errors.append(f"QK{i} read K slot holding {m.kslot[s]}")
-            if i > 0 and not (m.s_buf == i - 1 and m.s_reads == 4):
-                m.errors.append(f"QK{i} overwrote S{m.s_buf} after {m.s_reads} reads")
+            if i >= m.n_s and not (m.s_buf[sb] == i - m.n_s and m.s_reads[sb] == 4):
+                m.errors.append(f"QK{i} overwrote S{m.s_buf[sb]} after {m.s_reads[sb]} reads")
 
-        def end(i=i, s=s):
+        def end(i=i, s=s, sb=sb):
             if m.kslot[s] != i:
                 m.errors.append(f"QK{i}: K slot changed under it ({m.kslot[s]})")
-            m.s_buf, m.s_reads = i, 0
+            m.s_buf[sb], m.s_reads[sb] = i, 0
         m.mma(m.lat(300, 600), start, end)
         m.commit(m.s_full[i & 1])
         m.commit(m.ke[s])
@@ -165,8 +168,8 @@ def pv_issuer(m):
     if m.n == 0:
         return
     for j in range(m.n):
-        pb = j % 3
-        yield wait(m.p_full[pb], j // 3)
+        pb = j % m.n_p
+        yield wait(m.p_full[pb], j // m.n_p)
         s = j % m.nsv
         yield wait(m.vf[s], j // m.nsv)
 
@@ -191,11 +194,12 @@ def pv_issuer(m):
 def softmax(m, q, g):
     for j in range(g, m.n, 2):
         yield wait(m.s_full[g], j >> 1)
-        if m.s_buf != j:
-            m.errors.append(f"softmax q{q} read S{m.s_buf} for tile {j}")
+        sb = j % m.n_s
+        if m.s_buf[sb] != j:
+            m.errors.append(f"softmax q{q} read S{m.s_buf[sb]} for tile {j}")
         yield ("delay", m.lat(100, 300) * m.slow)
-        m.s_reads += 1
-        m.s_free.arrive()
+        m.s_reads[sb] += 1
+        m.s_free[sb].arrive()
         if j > 0:
             yield wait(m.m_ready[q][g ^ 1], (j - 1) >> 1)
             if m.mref.get((q, g ^ 1)) != j - 1:
@@ -203,16 +207,16 @@ def softmax(m, q, g):
         if j + 1 < m.n:
             m.mref[(q, g)] = j
             m.m_ready[q][g].arrive()
-        pb = j % 3
-        if j >= 3:
-            yield wait(m.pv_done[pb], (j - 3) // 3)
-            if m.pv_done_count < j - 2:
-                m.errors.append(f"P{j} written before PV{j - 3} finished")
+        pb = j % m.n_p
+        if j >= m.n_p:
+            yield wait(m.pv_done[pb], (j - m.n_p) // m.n_p)
+            if m.pv_done_count < j - m.n_p + 1:
+                m.errors.append(f"P{j} written before PV{j - m.n_p} finished")
         yield ("delay", m.lat(400, 2000) * m.slow)
         cur = m.p_buf[pb]
         m.p_buf[pb] = (j, (cur[1] + 1) if cur and cur[0] == j else 1)
         if j > 0 and m.rng.random() < m.p_rescale:
-            yield wait(m.pv_done[(j - 1) % 3], (j - 1) // 3)
+            yield wait(m.pv_done[(j - 1) % m.n_p], (j - 1) // m.n_p)
             if m.pv_done_count < j or m.pv_started >= j:
                 m.errors.append(f"O rescale at tile {j}: PV done {m.pv_done_count}, started {m.pv_started}")
             yield ("delay", m.lat(100, 400))
@@ -223,7 +227,8 @@ def softmax(m, q, g):
             m.errors.append(f"epilogue after {m.pv_done_count} of {m.n} PVs")
 
 
-CONFIGS = [(4, 4), (2, 2)]   # K / V ring slots at d = 64 and d = 128
+# K / V ring slots, TMEM score buffers, TMEM P buffers
+CONFIGS = [(4, 4, 1, 3), (2, 2, 1, 3), (4, 4, 2, 2), (2, 2, 2, 2), (4, 4, 1, 2)]
 
 
 @pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 8, 13])
@@ -232,7 +237,7 @@ def test_forward_schedule_finishes_without_aliasing(n, slots):
     for seed in range(20):
         for slow, v_lat in ((0.3, (200, 3000)), (1.0, (200, 3000)), (3.0, (200, 3000)),
                             (1.0, (3000, 9000))):
-            m = Fwd(n, slots[0], slots[1], seed, slow=slow, v_lat=v_lat)
+            m = Fwd(n, slots[0], slots[1], seed, slow=slow, v_lat=v_lat, n_s=slots[2], n_p=slots[3])
             roles = [k_producer(m), v_producer(m), qk_issuer(m), pv_issuer(m)]
             roles += [softmax(m, q, g) for q in range(4) for g in range(2)]
             assert m.run(roles), f"deadlock n={n} slots={slots} seed={seed}"
@@ -245,8 +250,8 @@ def test_model_detects_a_planted_mistake():
         for j in range(g, m.n, 2):
             yield wait(m.s_full[g], j >> 1)
             yield ("delay", m.lat(100, 300))
-            m.s_reads += 1
-            m.s_free.arrive()
+            m.s_reads[0] += 1
+            m.s_free[0].arrive()
             if j > 0:
                 yield wait(m.m_ready[q][g ^ 1], (j - 1) >> 1)
             if j + 1 < m.n:

@@ -32,3 +32,32 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     o_ref, lse_ref = oracle.attn_ref(q, k, v, 0.125, True, None)
     compare(o, lse, o_ref, lse_ref, "after timeout")
     assert fa_get_device_status() == FA_OK
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+def test_forward_wait_limit_runs_out_and_context_survives(d, causal):
+    # The forward kernel itself with a wait limit of a few cycles: some pipeline
+    # wait runs out, every role of that CTA stops after its own copies and MMAs
+    # have landed, and the call reports FA_ERR_DEVICE_TIMEOUT.  The context must
+    # stay usable: a normal call afterwards passes parity and leaves the status clean.
+    import torch
+    from io_aware_exact_24_b200 import (FA_ERR_DEVICE_TIMEOUT, FA_OK, fa_get_device_status,
+                                        fa_selftest_fwd_timeout)
+    from fa_testutil import to_device_bf16
+    assert fa_get_device_status() == FA_OK
+    B, H, N = 2, 4, 1000
+    q = normal_bf16((B, H, N, d), 6 + d, 0)
+    k = normal_bf16((B, H, N, d), 6 + d, 1)
+    v = normal_bf16((B, H, N, d), 6 + d, 2)
+    tq, tk, tv = to_device_bf16(q), to_device_bf16(k), to_device_bf16(v)
+    o = torch.empty_like(tq)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    for _ in range(2):
+        st = fa_selftest_fwd_timeout(tq, tk, tv, o, lse, B, H, N, N, d, scale, causal, 2)
+        assert st == FA_ERR_DEVICE_TIMEOUT
+        assert fa_get_device_status() == FA_OK      # read and cleared by the call
+    o2, lse2 = run_fa(q, k, v, scale, causal, None)
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, scale, causal, None)
+    compare(o2, lse2, o_ref, lse_ref, f"after forward timeout d={d}")
+    assert fa_get_device_status() == FA_OK

@@ -110,28 +110,34 @@ def check(o, lse, o_ref, lse_ref, bound, what):
     return ratio, lse_err
 
 
-def _inputs(B, H, Nq, Nk, seed, sigma=1.0):
-    q8, qd = normal_e4m3((B, H, Nq, 128), seed, 0, sigma)
-    k8, kd = normal_e4m3((B, H, Nk, 128), seed, 1, sigma)
-    v8, vd = normal_e4m3((B, H, Nk, 128), seed, 2, sigma)
+def _inputs(B, H, Nq, Nk, seed, sigma=1.0, d=128):
+    q8, qd = normal_e4m3((B, H, Nq, d), seed, 0, sigma)
+    k8, kd = normal_e4m3((B, H, Nk, d), seed, 1, sigma)
+    v8, vd = normal_e4m3((B, H, Nk, d), seed, 2, sigma)
     return q8, k8, v8, qd, kd, vd
 
 
 CASES = [
-    # B, H, Nq, Nk, causal, key_lens
-    (1, 4, 1000, 1000, True, None),       # 8 tiles, ragged tail of 104
-    (2, 2, 300, 900, False, [900, 200]),  # key padding
-    (1, 2, 400, 150, True, None),         # leading rows see no key
-    (2, 3, 129, 257, True, None),         # one row past a tile, ragged keys
-    (2, 2, 256, 384, False, [0, 384]),    # a sequence with no keys
+    # B, H, Nq, Nk, causal, key_lens, d
+    (1, 4, 1000, 1000, True, None, 128),       # 8 tiles, ragged tail of 104
+    (2, 2, 300, 900, False, [900, 200], 128),  # key padding
+    (1, 2, 400, 150, True, None, 128),         # leading rows see no key
+    (2, 3, 129, 257, True, None, 128),         # one row past a tile, ragged keys
+    (2, 2, 256, 384, False, [0, 384], 128),    # a sequence with no keys
+    # d = 64: rows of 64 one-byte codes, 64-byte swizzled tiles
+    (1, 4, 1000, 1000, True, None, 64),
+    (2, 2, 300, 900, False, [900, 200], 64),
+    (1, 2, 400, 150, True, None, 64),
+    (2, 3, 129, 257, True, None, 64),
+    (2, 2, 256, 384, False, [0, 384], 64),
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
 def test_fp8_matches_oracle_within_the_derived_bound(case):
-    B, H, Nq, Nk, causal, kl = case
-    scale = float(np.float32(1 / np.sqrt(128)))
-    q8, k8, v8, qd, kd, vd = _inputs(B, H, Nq, Nk, 900 + Nq + Nk)
+    B, H, Nq, Nk, causal, kl, d = case
+    scale = float(np.float32(1 / np.sqrt(d)))
+    q8, k8, v8, qd, kd, vd = _inputs(B, H, Nq, Nk, 900 + Nq + Nk + d, d=d)
     kl_arr = None if kl is None else np.array(kl, np.int32)
     o, lse = run_fp8(q8, k8, v8, scale, qd, kd, vd, causal, kl_arr)
     o_ref, lse_ref = oracle.attn_ref_e4m3(q8, k8, v8, scale, qd, kd, vd, causal, kl_arr)
@@ -148,14 +154,16 @@ def test_fp8_matches_oracle_within_the_derived_bound(case):
     print(f"{case}: max |dO|/bound {ratio:.3f}, max|dLSE| {lse_err:.2e}")
 
 
-def test_fp8_without_keys_gives_masked_rows():
-    q8, k8, v8, qd, kd, vd = _inputs(1, 2, 200, 1, 31)
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_without_keys_gives_masked_rows(d):
+    q8, k8, v8, qd, kd, vd = _inputs(1, 2, 200, 1, 31, d=d)
     o, lse = run_fp8(q8, k8[:, :, :0], v8[:, :, :0], 0.088, qd, kd, vd, False)
     assert np.all(o == 0) and not np.signbit(o).any() and np.all(np.isneginf(lse))
 
 
-def test_fp8_is_deterministic():
-    q8, k8, v8, qd, kd, vd = _inputs(1, 2, 600, 700, 41)
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_is_deterministic(d):
+    q8, k8, v8, qd, kd, vd = _inputs(1, 2, 600, 700, 41, d=d)
     a = run_fp8(q8, k8, v8, 0.088, qd, kd, vd, True)
     b = run_fp8(q8, k8, v8, 0.088, qd, kd, vd, True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
@@ -169,10 +177,11 @@ def test_fp8_v_descale_multiplies_o():
     assert np.array_equal(o2, o1 * 0.25) and np.array_equal(l1, l2)
 
 
-def test_fp8_full_size_sampled_rows():
-    """causal_8000_d128 at full size (B2 H32 N8000), in the launch configuration the
+@pytest.mark.parametrize("name", ["causal_8000_d128", "long_16k_d64"])
+def test_fp8_full_size_sampled_rows(name):
+    """The two long workloads at full size, in the launch configuration the
     benchmark times; sampled rows against the oracle's row entry point."""
-    w = WORKLOADS["causal_8000_d128"]
+    w = WORKLOADS[name]
     x = make_inputs_fp8(w)
     o, lse = run_fp8(x["q8"], x["k8"], x["v8"], w.scale, x["q_descale"], x["k_descale"],
                      x["v_descale"], w.causal)
@@ -189,12 +198,12 @@ def test_fp8_full_size_sampled_rows():
     for n, r in enumerate(rows):
         bh, i = divmod(int(r), w.Nq)
         b, h = divmod(bh, w.H)
-        vis = (np.arange(w.Nk) <= i + (w.Nk - w.Nq))[None, :]
+        vis = ((np.arange(w.Nk) <= i + (w.Nk - w.Nq)) | (not w.causal))[None, :]
         qf = oracle.e4m3_to_f64(x["q8"][b, h, i:i + 1])
         kf = oracle.e4m3_to_f64(x["k8"][b, h])
         vf = oracle.e4m3_to_f64(x["v8"][b, h]) * np.float64(np.float32(x["v_descale"]))
         bound[n] = bound_rows(qf, kf, vf, s_eff, vis, o_ref[n:n + 1])[0]
-    ratio, lse_err = check(o_f, l_f, o_ref, lse_ref, bound, "causal_8000_d128 e4m3")
+    ratio, lse_err = check(o_f, l_f, o_ref, lse_ref, bound, f"{name} e4m3")
     print(f"full size: max |dO|/bound {ratio:.3f}, max|dLSE| {lse_err:.2e}")
 
 

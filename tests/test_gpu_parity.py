@@ -1,8 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
 
-Small and medium problems are compared element by element; the two
-full-size long-sequence workloads are compared on sampled rows the oracle
-evaluates one by one, plus properties that hold at any size.
+All five workloads are compared element by element over every output row at
+their full sizes (the two long ones cost the oracle about half a minute each
+on the host cores), plus properties that hold at any size.
 """
 import numpy as np
 import pytest
@@ -40,30 +40,23 @@ def test_workload_full_compare(name):
     print(f"{name}: max|dO|={errs[0]:.3e} relF={errs[1]:.3e} max|dLSE|={errs[2]:.3e}")
 
 
-def _sample_rows(w, rng, per_head=12):
-    rows = []
-    edges = [0, 1, 127, 128, 255, 256, w.Nq - 129, w.Nq - 128, w.Nq - 65, w.Nq - 64, w.Nq - 2,
-             w.Nq - 1]
-    for bh in range(w.B * w.H):
-        pick = set(i for i in edges if 0 <= i < w.Nq)
-        pick.update(rng.integers(0, w.Nq, size=per_head).tolist())
-        rows += [bh * w.Nq + i for i in sorted(pick)]
-    return np.array(rows, np.int64)
-
-
 @pytest.mark.parametrize("name", ["long_16k_d64", "causal_8000_d128"])
-def test_workload_full_size_sampled_rows(name):
+def test_workload_full_size_every_row(name):
+    # the two long workloads at full size, in the launch configuration bench.py
+    # times, against the oracle on every row (per-row S and P keep host memory bounded)
     w = WORKLOADS[name]
     x = make_inputs(w)
     o, lse = run_fa(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
     assert np.isfinite(o).all() and np.isfinite(lse).all()
-    rows = _sample_rows(w, np.random.default_rng(123))
-    o_ref, lse_ref = oracle.attn_ref_rows(x["q"], x["k"], x["v"], w.scale, rows, w.causal,
-                                          x["key_lens"])
-    errs = compare(o.reshape(-1, w.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, name)
-    print(f"{name} ({rows.size} rows): max|dO|={errs[0]:.3e} relF={errs[1]:.3e} "
+    o_ref, lse_ref = oracle.attn_ref(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    errs = compare(o, lse, o_ref, lse_ref, name)
+    print(f"{name} (all {w.B * w.H * w.Nq} rows): max|dO|={errs[0]:.3e} relF={errs[1]:.3e} "
           f"max|dLSE|={errs[2]:.3e}")
-    # properties at full size: |O| is bounded by max|V| (convex combination of V rows)
+    # per (b, h) as well: no head may hide a larger relative error inside the total
+    num = np.linalg.norm((o - o_ref).reshape(w.B * w.H, -1), axis=1)
+    den = np.linalg.norm(o_ref.reshape(w.B * w.H, -1), axis=1)
+    assert (num / den).max() <= 4e-3
+    # |O| is bounded by max|V| (each row is a convex combination of V rows)
     vmax = np.abs(bf16_bits_to_f32(x["v"])).max()
     assert np.abs(o).max() <= vmax * (1 + 2**-7)
 

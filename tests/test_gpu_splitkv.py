@@ -115,3 +115,45 @@ def test_splitkv_deterministic_bitwise():
     a = run_splitkv(q, k, v, 0.09, False, None, 9)
     b = run_splitkv(q, k, v, 0.09, False, None, 9)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_splitkv_decode_64k_h8_benched_split():
+    # decode_64k_h8_d128 at full size, in the configuration bench.py times: the
+    # heuristic splits it (8 query blocks cannot fill the GPU), every row compared
+    from io_aware_exact_24_b200 import fa_splitkv_num_splits
+    w = DECODE_WORKLOADS["decode_64k_h8_d128"]
+    ns = fa_splitkv_num_splits(w.B, w.H, w.Nq, w.Nk)
+    assert ns > 1
+    x = make_inputs(w)
+    o, lse, guards = run_splitkv(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"], "auto")
+    assert guards, "wrote outside O / LSE"
+    o_ref, lse_ref = oracle.attn_ref(x["q"], x["k"], x["v"], w.scale, w.causal, x["key_lens"])
+    errs = compare(o, lse, o_ref, lse_ref, w.name)
+    print(f"{w.name} ({ns} ranges): max|dO|={errs[0]:.3e} relF={errs[1]:.3e} "
+          f"max|dLSE|={errs[2]:.3e}")
+
+
+@pytest.mark.parametrize("S,d,causal", [(2, 64, False), (37, 128, False), (256, 64, True),
+                                        (97, 128, True)])
+def test_splitkv_forced_many_ranges_long_keys(S, d, causal):
+    # N_k >= 32K with a ragged tail (313 K/V tiles), cut into up to 256 ranges of
+    # one or two tiles; a few query rows per head (causal: the last rows, which see
+    # nearly every key)
+    B, H, Nq, Nk = 1, 3, 3, 40000
+    seed = 900 + S + d
+    q = normal_bf16((B, H, Nq, d), seed, 0)
+    k = normal_bf16((B, H, Nk, d), seed, 1)
+    v = normal_bf16((B, H, Nk, d), seed, 2)
+    scale = 1.0 / np.sqrt(d)
+    o, lse, guards = run_splitkv(q, k, v, scale, causal, None, S)
+    assert guards, "wrote outside O / LSE"
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, scale, causal, None)
+    compare(o, lse, o_ref, lse_ref, f"S={S} d={d} causal={causal}")
+
+
+def test_splitkv_num_splits_uses_the_device_sm_count():
+    import torch
+    from io_aware_exact_24_b200 import fa_splitkv_num_splits
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # one query row, one head and a million keys: one range per SM
+    assert fa_splitkv_num_splits(1, 1, 1, 1 << 20) == min(sms, 256)
