@@ -16,6 +16,13 @@
 #include "fa.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
+#include "fa_fwd_persist.cuh"
+
+// Dense forward launches use the persistent kernel (fa_fwd_persist.cuh); 0 keeps
+// one CTA per query block to the end (the split-KV and packed modes always do).
+#ifndef FA_PERSISTENT
+#define FA_PERSISTENT 1
+#endif
 
 namespace {
 
@@ -37,6 +44,8 @@ constexpr long long kHeadGroupL2Bytes = (long long)FA_HEAD_GROUP_MB << 20;
 // below this many query blocks per (b, h) the per-CTA fixed cost dominates and
 // the plain order measured faster (GPT-2-sized causal problems, N = 1024)
 constexpr unsigned kHeadGroupMinBlocks = 32;
+// Longest K/V walk (tiles of 128 keys) for which the dense forward uses persistent CTAs.
+constexpr int kPersistMaxTiles = 16;
 constexpr int kMaxDevices = 64;
 // largest relative-position radius of a bias table (2^30: the table's
 // 2R+1 entries and every clamped index stay within int range)
@@ -63,8 +72,26 @@ EncodeTiledFn encoder() {
 struct DeviceState {
     std::once_flag once;
     int status = FA_OK;
+    int num_sms = 148;   // multiProcessorCount, read once
 };
 DeviceState g_dev[kMaxDevices];
+
+// Shared-memory limit of the persistent dense kernels of one head dim and input type.
+template <int D, bool kF8>
+cudaError_t set_persist_smem() {
+    const int bytes = fa::PersistCfg<D, kF8>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasNone>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (!kF8) {
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasSlopes>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasTable>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    }
+    return e;
+}
 
 // Per device, once: check the architecture and raise the kernels' shared-memory limit.
 int prepare_device(int dev) {
@@ -82,6 +109,9 @@ int prepare_device(int dev) {
             st.status = FA_ERR_UNSUPPORTED;
             return;
         }
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+            st.num_sms = sms;
         e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  fa::Cfg<64>::kSmemBytes);
         if (e == cudaSuccess)
@@ -117,6 +147,12 @@ int prepare_device(int dev) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, false, fa::kBiasTable>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+#if FA_PERSISTENT
+        if (e == cudaSuccess) e = set_persist_smem<64, false>();
+        if (e == cudaSuccess) e = set_persist_smem<128, false>();
+        if (e == cudaSuccess) e = set_persist_smem<64, true>();
+        if (e == cudaSuccess) e = set_persist_smem<128, true>();
+#endif
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      fa::BwdCfg<64>::kSmemBytes);
@@ -174,6 +210,11 @@ bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, 
                const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                span == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+__global__ void zero_ints_kernel(int* p, int n) {
+    const int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    if (i < n) p[i] = 0;
 }
 
 // Split-KV: partial results and per-block arrival counters in the workspace.
@@ -288,6 +329,31 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         const long long hb = (long long)H * B;
         p.head_group = (int)(hg < 1 ? 1 : (hg > hb ? hb : hg));
     }
+#if FA_PERSISTENT
+    // Dense launches with more query blocks than SMs and at most
+    // kPersistMaxTiles K/V tiles per block run persistent CTAs that take over the
+    // blocks not yet started: a block then costs about 1 us less of fixed time
+    // (next Q and first S prefetched under this block's tail, no CTA start), but
+    // the steady state is about 5 % slower per tile, so long blocks keep one CTA
+    // per block (measured: padded 16x16x512 d64 +13 %, causal 8x12x1024 d64 +2 %,
+    // 1x16x16384 d64 -4 %, causal 2x32x8000 d128 -5 %).
+    int dev = 0;
+    const bool persist = sp.num_splits <= 0 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 &&
+                         dev < kMaxDevices && (long long)num_m * H * B > g_dev[dev].num_sms &&
+                         (N_k + fa::kBlockN - 1) / fa::kBlockN <= kPersistMaxTiles;
+    if (persist) {
+        dim3 grid(num_m, (unsigned)H, (unsigned)B);
+        const int smem = fa::PersistCfg<D, kF8>::kSmemBytes;
+        if (bias.mode == fa::kBiasSlopes)
+            fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasSlopes><<<grid, fa::kNumThreads, smem, stream>>>(tq, tk, tv, p);
+        else if (bias.mode == fa::kBiasTable)
+            fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasTable><<<grid, fa::kNumThreads, smem, stream>>>(tq, tk, tv, p);
+        else
+            fa::fa_fwd_persist_kernel<D, kF8, fa::kBiasNone><<<grid, fa::kNumThreads, smem, stream>>>(tq, tk, tv, p);
+        const cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (persistent)", e);
+    }
+#endif
     if constexpr (kF8) {
         dim3 grid(num_m, (unsigned)H, (unsigned)B);
         fa::fa_fwd_sm100_kernel<D, false, false, true>
@@ -309,9 +375,13 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         const cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
     }
-    // the arrival counters start at zero (the workspace has no required contents)
-    cudaError_t e = cudaMemsetAsync(sp.counter, 0, sizeof(int) * (size_t)num_m * H * B, stream);
-    if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync (split-KV counters)", e);
+    // the arrival counters start at zero (the workspace has no required contents);
+    // a kernel on the same engine as the next launch, not a memset operation,
+    // which measured about 15 us of stream time on decode-sized calls
+    const int n_counters = (int)((size_t)num_m * H * B);
+    zero_ints_kernel<<<(unsigned)((n_counters + 255) / 256), 256, 0, stream>>>(sp.counter, n_counters);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kernel launch (split-KV counters)", e);
     dim3 grid(num_m * (unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
     fa::fa_fwd_sm100_kernel<D, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     e = cudaGetLastError();

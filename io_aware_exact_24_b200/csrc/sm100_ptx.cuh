@@ -102,6 +102,37 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
+// ---------------------------------------------------------------- cluster launch control
+// Ask the hardware scheduler to cancel the launch of a CTA of this grid that
+// has not started yet; the 16-byte response lands at `resp` (shared memory,
+// 16-byte aligned) and completes 16 transaction bytes on `bar` (the caller
+// posts the expect-tx).  One request may be in flight per CTA.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+            resp),
+        "r"(bar)
+        : "memory");
+}
+// Decode a response: true if a CTA was cancelled (its work now belongs to the
+// caller), with that CTA's blockIdx in x, y, z.
+__device__ __forceinline__ bool clc_query(uint32_t resp, int& x, int& y, int& z) {
+    uint32_t ok, ux, uy, uz;
+    asm volatile(
+        "{\n\t.reg .b128 h;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 h, [%4];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, h;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, %2, %3, _}, h;\n\t}"
+        : "=r"(ok), "=r"(ux), "=r"(uy), "=r"(uz)
+        : "r"(resp)
+        : "memory");
+    x = (int)ux;
+    y = (int)uy;
+    z = (int)uz;
+    return ok != 0;
+}
+
 // ---------------------------------------------------------------- register re-balancing
 // Per-warpgroup register budget change; every warp of the warpgroup must execute it.
 template <uint32_t N>

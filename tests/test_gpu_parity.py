@@ -100,6 +100,27 @@ def test_edge_cases(case):
     compare(o, lse, o_ref, lse_ref, str(case))
 
 
+MANY_BLOCKS = [
+    # grids several times the SM count: a running CTA takes over blocks that
+    # have not started (B, H, Nq, Nk, d, causal, key_lens)
+    (3, 40, 700, 700, 64, True, [700, 0, 333]),
+    (2, 48, 520, 600, 128, False, [600, 77]),
+    (4, 30, 1000, 1000, 128, True, None),
+]
+
+
+@pytest.mark.parametrize("case", MANY_BLOCKS, ids=[str(c[:6]) for c in MANY_BLOCKS])
+def test_more_blocks_than_sms(case):
+    B, H, Nq, Nk, d, causal, kl = case
+    q, k, v = _rand(B, H, Nq, Nk, d, 91 + Nq + d)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    out = {}
+    o, lse = run_fa(q, k, v, 1.0 / np.sqrt(d), causal, kl_arr, o_guard=4096, out=out)
+    assert out["guards_ok"], "wrote outside O / LSE"
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, 1.0 / np.sqrt(d), causal, kl_arr)
+    compare(o, lse, o_ref, lse_ref, str(case))
+
+
 def test_empty_problems_touch_nothing():
     import torch
     from io_aware_exact_24_b200 import fa_fwd
