@@ -212,6 +212,21 @@ bool encode_bhnd(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The backward's fp32 dQ accumulator [B*H, N, d] as a 3-D tensor for tensor reduces:
+// boxes of 32 columns x 32 rows (one warp's rows), 128-byte swizzle; rows past N
+// (a ragged last query tile) lie outside the tensor and are skipped.
+bool encode_dq_acc(CUtensorMap* map, float* ptr, int BH, int N, int d) {
+    EncodeTiledFn enc = encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 __global__ void zero_ints_kernel(int* p, int n) {
     const int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
     if (i < n) p[i] = 0;
@@ -482,9 +497,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync", e);
     }
     if (N_k > 0 && N_q > 0) {
-        CUtensorMap tq, tk, tv, tdo;
+        CUtensorMap tq, tk, tv, tdo, tdq;
         if (!encode_bhnd(&tq, q, B, H, N_q, D) || !encode_bhnd(&tk, k, B, H, N_k, D) ||
-            !encode_bhnd(&tv, v, B, H, N_k, D) || !encode_bhnd(&tdo, dout, B, H, N_q, D)) {
+            !encode_bhnd(&tv, v, B, H, N_k, D) || !encode_bhnd(&tdo, dout, B, H, N_q, D) ||
+            !encode_dq_acc(&tdq, dq_acc, B * H, N_q, D)) {
             snprintf(t_last_error, sizeof t_last_error, "cuTensorMapEncodeTiled failed");
             return FA_ERR_CUDA;
         }
@@ -504,7 +520,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         p.causal = causal ? 1 : 0;
         p.wait_limit = kWaitLimitCycles;
         dim3 grid((unsigned)((N_k + 127) / 128), (unsigned)H, (unsigned)B);
-        fa::fa_bwd_sm100_kernel<D><<<grid, fa::kBwdThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+        fa::fa_bwd_sm100_kernel<D><<<grid, fa::kBwdThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail("kernel launch (backward)", e);
     }

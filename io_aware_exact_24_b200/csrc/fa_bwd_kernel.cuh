@@ -15,7 +15,7 @@
 // Layout (one CTA per 128-key block of one (b, h); it walks the query tiles that
 // can see its keys):
 //  * warp 0 (one lane): TMA loads of K_j and V_j once, then Q_i and dO_i per
-//    query tile (kStages slots);
+//    query tile (Q and dO in rings of their own: kStagesQ / kStagesO slots);
 //  * warp 1 (one lane): the five tcgen05 MMAs of a tile --
 //      S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T     (M = 128 keys, N = 128 queries)
 //      dV  += P^T dO_i    and  dK  += dS^T Q_i       (A = P^T / dS^T from TMEM)
@@ -63,16 +63,24 @@ struct BwdCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kBoxes = D / 64;
     static constexpr int kTileBytes = 128 * D * 2;
-    static constexpr int kStages = (D == 64) ? 2 : 1;                // Q / dO slots
+    // Q and dO slots: two of each at d = 64, one of each at d = 128 (the room a
+    // second pair would take holds half of the dQ staging there)
+    static constexpr int kStagesQ = (D == 64) ? 2 : 1;
+    static constexpr int kStagesO = (D == 64) ? 2 : 1;
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKOff + kTileBytes;
-    static constexpr int kQOff = kVOff + kTileBytes;                  // [stage]
-    static constexpr int kDOOff = kQOff + kStages * kTileBytes;       // [stage]
-    static constexpr int kDSOff = kDOOff + kStages * kTileBytes;      // dS^T: 2 boxes of 64 queries
-    static constexpr int kRowOff = kDSOff + 2 * kSwizzleBoxBytes;     // [2][lse2 x128 | D x128] fp32
+    static constexpr int kQOff = kVOff + kTileBytes;                  // [kStagesQ]
+    static constexpr int kDOOff = kQOff + kStagesQ * kTileBytes;      // [kStagesO]
+    static constexpr int kDSOff = kDOOff + kStagesO * kTileBytes;     // dS^T: 2 boxes of 64 queries
+    // dQ staging for the tensor reduce (fp32, boxes of 32 columns x 128 rows, 128-byte
+    // swizzle): box (g, 0) of compute-warp half g is dS^T box g (free between the dQ
+    // product and the next tile's dS^T); at d = 128 box (g, 1) is extra box g here
+    static constexpr int kDQ2Off = kDSOff + 2 * kSwizzleBoxBytes;
+    static constexpr int kRowOff = kDQ2Off + (D == 128 ? 2 * kSwizzleBoxBytes : 0);   // [2][lse2 x128 | D x128] fp32
     static constexpr int kBarOff = kRowOff + 2 * 256 * 4;
-    // barriers: kv_full, q_full[S], q_empty[S], s_full, p_full, dq_full, s_free, drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 5;
+    // barriers: kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], s_full,
+    // p_full, dq_full, s_free, drain
+    static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesO + 5;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
@@ -112,7 +120,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = smem_addr(smem_raw);
@@ -122,12 +130,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar = [&](int i) { return base + C::kBarOff + 8u * (uint32_t)i; };
     const uint32_t bar_kv = bar(0);
     auto bar_q_full = [&](int s) { return bar(1 + s); };
-    auto bar_q_empty = [&](int s) { return bar(1 + C::kStages + s); };
-    const uint32_t bar_s_full = bar(1 + 2 * C::kStages);
-    const uint32_t bar_p_full = bar(2 + 2 * C::kStages);
-    const uint32_t bar_dq_full = bar(3 + 2 * C::kStages);
-    const uint32_t bar_s_free = bar(4 + 2 * C::kStages);
-    const uint32_t bar_drain = bar(5 + 2 * C::kStages);
+    auto bar_q_empty = [&](int s) { return bar(1 + C::kStagesQ + s); };
+    auto bar_o_full = [&](int s) { return bar(1 + 2 * C::kStagesQ + s); };
+    auto bar_o_empty = [&](int s) { return bar(1 + 2 * C::kStagesQ + C::kStagesO + s); };
+    constexpr int kB0 = 1 + 2 * C::kStagesQ + 2 * C::kStagesO;
+    const uint32_t bar_s_full = bar(kB0);
+    const uint32_t bar_p_full = bar(kB0 + 1);
+    const uint32_t bar_dq_full = bar(kB0 + 2);
+    const uint32_t bar_s_free = bar(kB0 + 3);
+    const uint32_t bar_drain = bar(kB0 + 4);
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
     float* const rows = reinterpret_cast<float*>(base_ptr + C::kRowOff);
@@ -155,9 +166,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (warp == kBwdProducerWarp && lane == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < C::kStagesQ; ++s) {
             mbar_init(bar_q_full(s), 1);
             mbar_init(bar_q_empty(s), 1);
+        }
+        for (int s = 0; s < C::kStagesO; ++s) {
+            mbar_init(bar_o_full(s), 1);
+            mbar_init(bar_o_empty(s), 1);
         }
         mbar_init(bar_s_full, 1);
         mbar_init(bar_p_full, kBwdComputeWarps);    // one arrival per compute warp
@@ -170,6 +185,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
+        prefetch_tensormap(&tm_dq);
     }
     if (warp == kBwdMmaWarp) {
         tmem_alloc(smem_addr(tmem_holder), 512);
@@ -192,25 +208,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             policy_evict_first());
             }
             bool ok = true;
-            int t = 0;
-            for (; t < n_t; ++t) {
-                const int s = t % C::kStages;
-                ok = wait_bounded(bar_q_empty(s), (uint32_t)(((t / C::kStages) & 1) ^ 1), abort_flag, p.wait_limit);
-                if (!ok) break;
-                mbar_arrive_expect_tx(bar_q_full(s), 2u * (uint32_t)C::kTileBytes);
+            int nq = 0, no = 0;   // Q and dO copies issued
+            for (int t = 0; t < n_t && ok; ++t) {
                 const int q0 = (i_lo + t) * 128;
-                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                    tma_load_4d(base + C::kQOff + s * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_q, bar_q_full(s),
+                const int sq = t % C::kStagesQ;
+                ok = wait_bounded(bar_q_empty(sq), (uint32_t)(((t / C::kStagesQ) & 1) ^ 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_q_full(sq), (uint32_t)C::kTileBytes);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(base + C::kQOff + sq * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_q, bar_q_full(sq),
                                 bx * 64, q0, h, b, pol_keep);
-                    tma_load_4d(base + C::kDOOff + s * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_do,
-                                bar_q_full(s), bx * 64, q0, h, b, pol_keep);
-                }
+                ++nq;
+                const int so = t % C::kStagesO;
+                ok = wait_bounded(bar_o_empty(so), (uint32_t)(((t / C::kStagesO) & 1) ^ 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_o_full(so), (uint32_t)C::kTileBytes);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(base + C::kDOOff + so * C::kTileBytes + bx * kSwizzleBoxBytes, &tm_do, bar_o_full(so),
+                                bx * 64, q0, h, b, pol_keep);
+                ++no;
             }
             // wind down: every copy issued lands before the CTA exits
             wait_own_work(bar_kv, 0, p.wait_limit);
-            if (!ok)
-                for (int c2 = (t > C::kStages ? t - C::kStages : 0); c2 < t; ++c2)
-                    wait_own_work(bar_q_full(c2 % C::kStages), (uint32_t)((c2 / C::kStages) & 1), p.wait_limit);
+            if (!ok) {
+                for (int c2 = (nq > C::kStagesQ ? nq - C::kStagesQ : 0); c2 < nq; ++c2)
+                    wait_own_work(bar_q_full(c2 % C::kStagesQ), (uint32_t)((c2 / C::kStagesQ) & 1), p.wait_limit);
+                for (int c2 = (no > C::kStagesO ? no - C::kStagesO : 0); c2 < no; ++c2)
+                    wait_own_work(bar_o_full(c2 % C::kStagesO), (uint32_t)((c2 / C::kStagesO) & 1), p.wait_limit);
+            }
         }
         __syncwarp();
     } else if (warp == kBwdMmaWarp) {
@@ -219,20 +244,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool ok = wait_bounded(bar_kv, 0, abort_flag, p.wait_limit);
             const uint32_t k_s = base + C::kKOff, v_s = base + C::kVOff, ds_s = base + C::kDSOff;
             for (int t = 0; t < n_t && ok; ++t) {
-                const int s = t % C::kStages;
-                ok = wait_bounded(bar_q_full(s), (uint32_t)((t / C::kStages) & 1), abort_flag, p.wait_limit);
+                const int sq = t % C::kStagesQ, so = t % C::kStagesO;
+                ok = wait_bounded(bar_q_full(sq), (uint32_t)((t / C::kStagesQ) & 1), abort_flag, p.wait_limit);
                 // the previous tile's dQ has been read out of the S columns
                 if (ok && t > 0) ok = wait_bounded(bar_s_free, (uint32_t)((t - 1) & 1), abort_flag, p.wait_limit);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t q_s = base + C::kQOff + s * C::kTileBytes;
-                const uint32_t do_s = base + C::kDOOff + s * C::kTileBytes;
+                const uint32_t q_s = base + C::kQOff + sq * C::kTileBytes;
+                const uint32_t do_s = base + C::kDOOff + so * C::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
                     const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
                     umma_ss(tmem + C::kColS, smem_desc_sw128(k_s + koff, 16, 1024), smem_desc_sw128(q_s + koff, 16, 1024),
                             C::kIdescST, kk > 0 ? 1u : 0u);
                 }
+                // dO_i may land after Q_i (its slot frees when the previous tile's dV is done)
+                ok = wait_bounded(bar_o_full(so), (uint32_t)((t / C::kStagesO) & 1), abort_flag, p.wait_limit);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
                     const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
@@ -250,13 +279,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             smem_desc_sw128(do_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
+                umma_commit(bar_o_empty(so));   // dO_i is no longer read
 #pragma unroll
                 for (int kk = 0; kk < 128 / 16; ++kk) {   // dK += dS^T Q
                     umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(kk * 8 + 32 * (kk / 4)),
                             smem_desc_sw128(q_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(bar_q_empty(s));   // Q_i and dO_i are no longer read
+                umma_commit(bar_q_empty(sq));   // Q_i is no longer read
 #pragma unroll
                 for (int kk = 0; kk < 128 / 16; ++kk) {   // dQ = dS K: 16 keys per step
                     umma_ss(tmem + C::kColS, smem_desc_sw128(ds_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024),
@@ -306,28 +336,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 continue;
             }
             tc_fence_after();
+            // this key row sees every query of the tile (no per-element mask)
+            const bool row_full = key_ok && (!p.causal || k <= i0 + off);
+            // the previous tile's dQ reduce (issued by this warp's lane 0) has read its
+            // staging, part of which is the dS^T box written below
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
 #pragma unroll 1
             for (int cb = 2 * g; cb < 2 * g + 2; ++cb) {   // queries 32cb .. 32cb+31
                 uint32_t su[32], du[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32u * cb, su);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32u * cb, du);
+                // the 32 queries' LSE (log2 units) and D, same for every lane: 16-byte
+                // shared-memory loads while the TMEM loads are in flight
+                float lq[32], dq[32];
+                {
+                    const uint32_t ra = smem_addr(rb + 32 * cb);
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        ld_shared_v4(ra + 16u * i4, lq[4 * i4], lq[4 * i4 + 1], lq[4 * i4 + 2], lq[4 * i4 + 3]);
+                        ld_shared_v4(ra + 512u + 16u * i4, dq[4 * i4], dq[4 * i4 + 1], dq[4 * i4 + 2], dq[4 * i4 + 3]);
+                    }
+                }
                 tmem_wait_ld();
                 uint32_t pw[16], dw[16];
+                const int qa0 = i0 + 32 * cb;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     reg_after_wait(su[e]);
                     reg_after_wait(su[e + 1]);
                     reg_after_wait(du[e]);
                     reg_after_wait(du[e + 1]);
-                    const int qa = i0 + 32 * cb + e;
-                    const bool v0 = key_ok && (!p.causal || k <= qa + off);
-                    const bool v1 = key_ok && (!p.causal || k <= qa + 1 + off);
-                    const float p0 = v0 ? ex2_approx(__uint_as_float(su[e]) * c - rb[32 * cb + e]) : 0.f;
-                    const float p1 = v1 ? ex2_approx(__uint_as_float(su[e + 1]) * c - rb[32 * cb + e + 1]) : 0.f;
-                    const float d0 = p0 * (__uint_as_float(du[e]) - rb[128 + 32 * cb + e]);
-                    const float d1 = p1 * (__uint_as_float(du[e + 1]) - rb[128 + 32 * cb + e + 1]);
+                    // log2-domain score minus LSE, then P = 2^x and dS = P (dP - D)
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[e]), __uint_as_float(su[e + 1])),
+                                                make_float2(c, c), make_float2(-lq[e], -lq[e + 1]));
+                    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+                    if (!row_full) {
+                        const bool v0 = key_ok && k <= qa0 + e + off;
+                        const bool v1 = key_ok && k <= qa0 + e + 1 + off;
+                        p0 = v0 ? p0 : 0.f;
+                        p1 = v1 ? p1 : 0.f;
+                    }
+                    const float2 ds = __fmul2_rn(make_float2(p0, p1),
+                                                 __fadd2_rn(make_float2(__uint_as_float(du[e]), __uint_as_float(du[e + 1])),
+                                                            make_float2(-dq[e], -dq[e + 1])));
                     pw[e >> 1] = pack_bf16x2(p0, p1);
-                    dw[e >> 1] = pack_bf16x2(d0, d1);
+                    dw[e >> 1] = pack_bf16x2(ds.x, ds.y);
                 }
                 // P^T over S^T's columns 16cb + 32g.., dS^T over dP^T's: inside the 64
                 // columns this warp has read (the other warp of the quadrant reads
@@ -358,26 +412,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 continue;
             }
             tc_fence_after();
-            const int q = i0 + r;
-#pragma unroll 1
-            for (int c2 = g * (D / 64); c2 < (g + 1) * (D / 64); ++c2) {   // this warp's half of dQ
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_off + C::kColS + 32u * c2, u);
+            {
+                uint32_t u[D / 2];   // this warp's half of dQ row i0 + r
+#pragma unroll
+                for (int c2 = 0; c2 < D / 64; ++c2)
+                    tmem_ld32(tmem + lane_off + C::kColS + 32u * (uint32_t)(g * (D / 64) + c2),
+                              *reinterpret_cast<uint32_t(*)[32]>(&u[32 * c2]));
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) reg_after_wait(u[i]);
-                if (q < p.Nq) {
-                    float* dst = p.dq_acc + (bh * (size_t)p.Nq + q) * D + 32 * c2;
+                for (int i = 0; i < D / 2; ++i) reg_after_wait(u[i]);
+                // dQ_i is in registers: the next tile's S^T may take its TMEM columns
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_s_free);
+                // stage row r of this warp's boxes (32 fp32 columns each, 128-byte rows,
+                // 16-byte chunk cc at cc ^ (r % 8)) and add them into the fp32
+                // accumulator with one tensor reduce per box: rows past N_q are outside
+                // the tensor and skipped
 #pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        red_add_v4(dst + 4 * v4, __uint_as_float(u[4 * v4]), __uint_as_float(u[4 * v4 + 1]),
-                                   __uint_as_float(u[4 * v4 + 2]), __uint_as_float(u[4 * v4 + 3]));
+                for (int c2 = 0; c2 < D / 64; ++c2) {
+                    const uint32_t box = base + (c2 == 0 ? C::kDSOff : C::kDQ2Off) + (uint32_t)(g * kSwizzleBoxBytes);
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const uint32_t a = box + (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(u[32 * c2 + 4 * cc]),
+                                     "r"(u[32 * c2 + 4 * cc + 1]), "r"(u[32 * c2 + 4 * cc + 2]),
+                                     "r"(u[32 * c2 + 4 * cc + 3])
+                                     : "memory");
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int c2 = 0; c2 < D / 64; ++c2) {
+                        const uint32_t box =
+                            base + (c2 == 0 ? C::kDSOff : C::kDQ2Off) + (uint32_t)(g * kSwizzleBoxBytes);
+                        tma_reduce_add_3d(&tm_dq, box + (uint32_t)(qd * 32 * 128), (g * (D / 64) + c2) * 32,
+                                          i0 + qd * 32, (int)bh);
+                    }
+                    bulk_commit_group();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_s_free);
         }
+        // every dQ reduce this warp issued has completed before the CTA exits
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
         // ------------------------------------------------------------ dV, dK -> bf16
         bool have = n_t > 0;
         if (have && ok) {

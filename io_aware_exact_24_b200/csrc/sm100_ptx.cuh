@@ -78,6 +78,15 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, uint32_t src,
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// 3-D tiled reduce-add shared -> global (fp32 elements added into the tensor;
+// elements outside the tensor are skipped), tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(m)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -281,6 +290,11 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Ties a register produced by tcgen05.ld to a point after tcgen05.wait::ld, so
 // the compiler cannot move its first use above the wait.
 __device__ __forceinline__ void reg_after_wait(uint32_t& x) { asm volatile("" : "+r"(x)); }
+
+// 16-byte shared-memory load of four floats (address in the shared window).
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, float& a, float& b, float& c, float& d) {
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(a), "=f"(b), "=f"(c), "=f"(d) : "r"(addr));
+}
 
 // ---------------------------------------------------------------- arithmetic
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -34,9 +34,10 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, n_t, stages, seed, warps=8):
+    def __init__(self, n_t, stages, seed, warps=8, stages_o=None):
         self.rng = random.Random(seed)
         self.n_t, self.S, self.W = n_t, stages, warps
+        self.SO = stages if stages_o is None else stages_o
         self.now = 0
         self.events = []          # (time, seq, callable)
         self.seq = 0
@@ -44,14 +45,19 @@ class Sim:
         self.kv = b("kv_full", 1)
         self.q_full = [b(f"q_full{s}", 1) for s in range(stages)]
         self.q_empty = [b(f"q_empty{s}", 1) for s in range(stages)]
+        self.o_full = [b(f"o_full{s}", 1) for s in range(self.SO)]
+        self.o_empty = [b(f"o_empty{s}", 1) for s in range(self.SO)]
         self.s_full, self.p_full = b("s_full", 1), b("p_full", warps)
         self.dq_full, self.s_free = b("dq_full", 1), b("s_free", warps)
         self.drain = b("drain", 1)
         # buffer contents: which tile's data they hold
-        self.slot = [None] * stages           # Q/dO slot -> tile
+        self.slot = [None] * stages           # Q slot -> tile
+        self.oslot = [None] * self.SO         # dO slot -> tile
         self.s_cols = None                    # S^T / P^T / dQ columns: ("S", t) / ("dQ", t)
         self.dp_cols = None                   # dP^T / dS^T columns
         self.ds_smem = None                   # dS^T in shared memory
+        self.stage = [None] * warps           # each warp's part of that buffer: ("dS", t) / ("dQ", t)
+        self.reading = [False] * warps        # a tensor reduce is still reading the warp's dQ staging
         self.tc_free_at = 0                   # tensor core busy until
         self.errors = []
 
@@ -134,6 +140,13 @@ def producer(sim):
             sim.slot[s] = t
             sim.q_full[s].arrive()
         sim.at(sim.lat(50, 600), land)
+        so = t % sim.SO
+        yield wait(sim.o_empty[so], t // sim.SO - 1)
+
+        def land_o(so=so, t=t):
+            sim.oslot[so] = t
+            sim.o_full[so].arrive()
+        sim.at(sim.lat(50, 600), land_o)
         yield ("delay", 1)
 
 
@@ -145,25 +158,37 @@ def issuer(sim):
         if t > 0:
             yield wait(sim.s_free, t - 1)
 
-        def mma12(t=t, s=s):
+        def mma1(t=t, s=s):
             if sim.slot[s] != t:
-                sim.errors.append(f"S/dP of tile {t} read slot holding {sim.slot[s]}")
-            sim.s_cols, sim.dp_cols = ("S", t), ("dP", t)
-        sim.mma(sim.lat(100, 300), mma12)
+                sim.errors.append(f"S of tile {t} read Q slot holding {sim.slot[s]}")
+            sim.s_cols = ("S", t)
+        sim.mma(sim.lat(50, 150), mma1)
+        so = t % sim.SO
+        yield wait(sim.o_full[so], t // sim.SO)
+
+        def mma2(t=t, so=so):
+            if sim.oslot[so] != t:
+                sim.errors.append(f"dP of tile {t} read dO slot holding {sim.oslot[so]}")
+            sim.dp_cols = ("dP", t)
+        sim.mma(sim.lat(50, 150), mma2)
         sim.commit(sim.s_full)
         yield wait(sim.p_full, t)
 
-        def mma34(t=t, s=s):
-            if sim.slot[s] != t:
-                sim.errors.append(f"dV/dK of tile {t} read slot holding {sim.slot[s]}")
-            if sim.s_cols != ("P", t) or sim.dp_cols != ("dS", t):
-                sim.errors.append(f"dV/dK of tile {t} read {sim.s_cols} {sim.dp_cols}")
-        sim.mma(sim.lat(100, 300), mma34)
+        def mma3(t=t, so=so):
+            if sim.oslot[so] != t or sim.s_cols != ("P", t):
+                sim.errors.append(f"dV of tile {t} read dO {sim.oslot[so]}, {sim.s_cols}")
+        sim.mma(sim.lat(50, 150), mma3)
+        sim.commit(sim.o_empty[so])
+
+        def mma4(t=t, s=s):
+            if sim.slot[s] != t or sim.dp_cols != ("dS", t):
+                sim.errors.append(f"dK of tile {t} read Q {sim.slot[s]}, {sim.dp_cols}")
+        sim.mma(sim.lat(50, 150), mma4)
         sim.commit(sim.q_empty[s])
 
         def mma5(t=t):
-            if sim.ds_smem != t:
-                sim.errors.append(f"dQ of tile {t} read dS^T of {sim.ds_smem}")
+            if sim.ds_smem != t or any(st != ("dS", t) for st in sim.stage):
+                sim.errors.append(f"dQ of tile {t} read dS^T of {sim.ds_smem} / {sim.stage}")
             sim.s_cols = ("dQ", t)
         sim.mma(sim.lat(50, 200), mma5)
         sim.commit(sim.dq_full)
@@ -182,6 +207,10 @@ def compute_warp(sim, w, rows_barrier):
         # when the reads end
         if sim.s_cols not in (("S", t), ("P", t)) or sim.dp_cols not in (("dP", t), ("dS", t)):
             sim.errors.append(f"warp {w} tile {t}: S/dP overwritten during the read")
+        # dS^T goes where this warp staged the previous tile's dQ: its reduce must be done reading
+        while sim.reading[w]:
+            yield ("delay", 10)
+        sim.stage[w] = ("dS", t)
         sim.s_cols, sim.dp_cols, sim.ds_smem = ("P", t), ("dS", t), t
         sim.p_full.arrive()
         yield wait(sim.dq_full, t)
@@ -191,6 +220,17 @@ def compute_warp(sim, w, rows_barrier):
         if sim.s_cols != ("dQ", t):
             sim.errors.append(f"warp {w} tile {t}: dQ overwritten during the read")
         sim.s_free.arrive()
+        # dQ staged in this warp's part of the dS^T buffer (the dQ product, its last
+        # reader, is done), then a tensor reduce reads it asynchronously
+        yield ("delay", sim.lat(20, 200))
+        sim.stage[w] = ("dQ", t)
+        sim.reading[w] = True
+
+        def read_done(w=w, t=t):
+            if sim.stage[w] != ("dQ", t):
+                sim.errors.append(f"warp {w}: dQ staging of tile {t} overwritten during the reduce")
+            sim.reading[w] = False
+        sim.at(sim.lat(100, 3000), read_done)
     if sim.n_t > 0:
         yield wait(sim.drain, 0)
 
@@ -211,10 +251,10 @@ def make_named_barrier(sim):
 
 
 @pytest.mark.parametrize("n_t", [1, 2, 3, 7])
-@pytest.mark.parametrize("stages", [1, 2])
+@pytest.mark.parametrize("stages", [(1, 1), (2, 2), (2, 1)])
 def test_backward_schedule_finishes_without_aliasing(n_t, stages):
     for seed in range(25):
-        sim = Sim(n_t, stages, seed)
+        sim = Sim(n_t, stages[0], seed, stages_o=stages[1])
         nb = make_named_barrier(sim)
         roles = [producer(sim), issuer(sim)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
         assert sim.run(roles), f"deadlock (n_t={n_t}, stages={stages}, seed={seed})"
@@ -234,7 +274,10 @@ def test_model_detects_a_planted_mistake():
             sim.mma(50, mma12)
             sim.commit(sim.s_full)
             yield wait(sim.p_full, t)
+            so = t % sim.SO
+            yield wait(sim.o_full[so], t // sim.SO)
             sim.mma(50, lambda: None)
+            sim.commit(sim.o_empty[so])
             sim.commit(sim.q_empty[s])
 
             def mma5(t=t):
@@ -250,6 +293,41 @@ def test_model_detects_a_planted_mistake():
         roles = [producer(sim), bad_issuer(sim)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
         ok = sim.run(roles)
         if not ok or sim.errors:
+            found = True
+            break
+    assert found
+
+
+def test_model_detects_a_missing_reduce_wait():
+    # a compute warp writes dS^T without waiting for its dQ reduce to read the staging
+    def bad_compute(sim, w, rows_barrier):
+        for t in range(sim.n_t):
+            yield from rows_barrier(t)
+            yield wait(sim.s_full, t)
+            yield ("delay", sim.lat(100, 800))
+            sim.stage[w] = ("dS", t)
+            sim.s_cols, sim.dp_cols, sim.ds_smem = ("P", t), ("dS", t), t
+            sim.p_full.arrive()
+            yield wait(sim.dq_full, t)
+            yield ("delay", sim.lat(50, 500))
+            sim.s_free.arrive()
+            sim.stage[w] = ("dQ", t)
+            sim.reading[w] = True
+
+            def read_done(w=w, t=t):
+                if sim.stage[w] != ("dQ", t):
+                    sim.errors.append("staging overwritten")
+                sim.reading[w] = False
+            sim.at(sim.lat(1000, 5000), read_done)
+        if sim.n_t > 0:
+            yield wait(sim.drain, 0)
+
+    found = False
+    for seed in range(25):
+        sim = Sim(5, 2, seed)
+        nb = make_named_barrier(sim)
+        roles = [producer(sim), issuer(sim)] + [bad_compute(sim, w, nb) for w in range(sim.W)]
+        if not sim.run(roles) or sim.errors:
             found = True
             break
     assert found
