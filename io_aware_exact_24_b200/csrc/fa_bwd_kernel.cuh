@@ -33,6 +33,8 @@
 // out records FA_ERR_DEVICE_TIMEOUT and the CTA winds down.
 #pragma once
 
+#include <type_traits>
+
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -338,6 +340,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             // this key row sees every query of the tile (no per-element mask)
             const bool row_full = key_ok && (!p.causal || k <= i0 + off);
+            // ... for every row of the warp, and no query row of the tile lies past N_q
+            const bool warp_full = __all_sync(0xffffffffu, row_full) && i0 + 128 <= p.Nq;
             // the previous tile's dQ reduce (issued by this warp's lane 0) has read its
             // staging, part of which is the dS^T box written below
             if (lane == 0) bulk_wait_group_read0();
@@ -361,28 +365,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_wait_ld();
                 uint32_t pw[16], dw[16];
                 const int qa0 = i0 + 32 * cb;
+                // one pair in four of the exponentials on the FMA pipe (MUFU is the
+                // busiest unit here), where every score of the warp is visible and
+                // finite (2^x is then the same up to rounding and a 2^-125 floor)
+                auto body = [&](auto emu_tag) {
+                    constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    reg_after_wait(su[e]);
-                    reg_after_wait(su[e + 1]);
-                    reg_after_wait(du[e]);
-                    reg_after_wait(du[e + 1]);
-                    // log2-domain score minus LSE, then P = 2^x and dS = P (dP - D)
-                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[e]), __uint_as_float(su[e + 1])),
-                                                make_float2(c, c), make_float2(-lq[e], -lq[e + 1]));
-                    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-                    if (!row_full) {
-                        const bool v0 = key_ok && k <= qa0 + e + off;
-                        const bool v1 = key_ok && k <= qa0 + e + 1 + off;
-                        p0 = v0 ? p0 : 0.f;
-                        p1 = v1 ? p1 : 0.f;
+                    for (int e = 0; e < 32; e += 2) {
+                        reg_after_wait(su[e]);
+                        reg_after_wait(su[e + 1]);
+                        reg_after_wait(du[e]);
+                        reg_after_wait(du[e + 1]);
+                        // log2-domain score minus LSE, then P = 2^x and dS = P (dP - D)
+                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(su[e]), __uint_as_float(su[e + 1])),
+                                                    make_float2(c, c), make_float2(-lq[e], -lq[e + 1]));
+                        float p0, p1;
+                        if (kEmu && (e & 6) == 6) {
+                            const float2 pe = exp2_fma2(x);
+                            p0 = pe.x;
+                            p1 = pe.y;
+                        } else {
+                            p0 = ex2_approx(x.x);
+                            p1 = ex2_approx(x.y);
+                        }
+                        if (!kEmu && !row_full) {
+                            const bool v0 = key_ok && k <= qa0 + e + off;
+                            const bool v1 = key_ok && k <= qa0 + e + 1 + off;
+                            p0 = v0 ? p0 : 0.f;
+                            p1 = v1 ? p1 : 0.f;
+                        }
+                        const float2 ds =
+                            __fmul2_rn(make_float2(p0, p1),
+                                       __fadd2_rn(make_float2(__uint_as_float(du[e]), __uint_as_float(du[e + 1])),
+                                                  make_float2(-dq[e], -dq[e + 1])));
+                        pw[e >> 1] = pack_bf16x2(p0, p1);
+                        dw[e >> 1] = pack_bf16x2(ds.x, ds.y);
                     }
-                    const float2 ds = __fmul2_rn(make_float2(p0, p1),
-                                                 __fadd2_rn(make_float2(__uint_as_float(du[e]), __uint_as_float(du[e + 1])),
-                                                            make_float2(-dq[e], -dq[e + 1])));
-                    pw[e >> 1] = pack_bf16x2(p0, p1);
-                    dw[e >> 1] = pack_bf16x2(ds.x, ds.y);
-                }
+                };
+                if (warp_full)
+                    body(std::true_type{});
+                else
+                    body(std::false_type{});
                 // P^T over S^T's columns 16cb + 32g.., dS^T over dP^T's: inside the 64
                 // columns this warp has read (the other warp of the quadrant reads
                 // the other 64), and after this warp read them
