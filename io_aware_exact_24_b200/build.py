@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_fwd_persist.cuh", "fa_bwd_kernel.cuh", "sm100_ptx.cuh",
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_fwd_persist.cuh", "fa_decode_kernel.cuh", "fa_bwd_kernel.cuh", "sm100_ptx.cuh",
                                                      "exp2_poly.cuh")] + [
     os.path.join(ROOT, "include", "fa.h")]
 OUT = os.path.join(PKG, "libfa_b200.so")

@@ -13,10 +13,13 @@
 #include <cstring>
 #include <mutex>
 
+#include <utility>
+
 #include "fa.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_fwd_persist.cuh"
+#include "fa_decode_kernel.cuh"
 
 // Dense forward launches use the persistent kernel (fa_fwd_persist.cuh); 0 keeps
 // one CTA per query block to the end (the split-KV and packed modes always do).
@@ -147,6 +150,12 @@ int prepare_device(int dev) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fa::fa_fwd_sm100_kernel<128, false, false, false, fa::kBiasTable>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Cfg<128>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_decode_splitkv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::DecCfg<64>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fa::fa_decode_splitkv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fa::DecCfg<128>::kSmemBytes);
 #if FA_PERSISTENT
         if (e == cudaSuccess) e = set_persist_smem<64, false>();
         if (e == cudaSuccess) e = set_persist_smem<128, false>();
@@ -228,8 +237,28 @@ bool encode_dq_acc(CUtensorMap* map, float* ptr, int BH, int N, int d) {
 }
 
 __global__ void zero_ints_kernel(int* p, int n) {
+    fa::pdl_launch_dependents();   // the split kernel touches the counters only after waiting
     const int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
     if (i < n) p[i] = 0;
+}
+
+// Launch a kernel that may start while the previous kernel of the stream (the
+// counters' zeroing) still runs; it waits for that kernel before its first use
+// of the counters (programmatic dependent launch).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Split-KV: partial results and per-block arrival counters in the workspace.
@@ -397,9 +426,18 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     zero_ints_kernel<<<(unsigned)((n_counters + 255) / 256), 256, 0, stream>>>(sp.counter, n_counters);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("kernel launch (split-KV counters)", e);
+    if (N_q == 1) {
+        // one query row: matrix-vector products, streamed on the CUDA cores
+        dim3 grid((unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
+        e = launch_dependent(fa::fa_decode_splitkv_kernel<D>, grid, dim3(fa::kDecThreads), fa::DecCfg<D>::kSmemBytes,
+                             stream, tk, tv, reinterpret_cast<const __nv_bfloat16*>(q), p);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (decode)", e);
+    }
     dim3 grid(num_m * (unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
-    fa::fa_fwd_sm100_kernel<D, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-    e = cudaGetLastError();
+    e = launch_dependent(fa::fa_fwd_sm100_kernel<D, true>, grid, dim3(fa::kNumThreads), fa::Cfg<D>::kSmemBytes, stream,
+                         tq, tk, tv, to, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV)", e);
     }
 }

@@ -358,6 +358,7 @@ __device__ __forceinline__ void split_merge(const FwdParams& p, uint8_t* flag_sm
     if (threadIdx.x == 0) {
         // every softmax thread fenced its own partial stores before the barrier
         // that preceded this arrival
+        pdl_wait_primary();   // the counters' zeroing kernel (it may still run: dependent launch)
         const int old = atomicAdd(p.split_counter + grp, 1);
         *flag = (old == n_split - 1) ? 1 : 0;
     }

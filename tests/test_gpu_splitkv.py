@@ -151,6 +151,25 @@ def test_splitkv_forced_many_ranges_long_keys(S, d, causal):
     compare(o, lse, o_ref, lse_ref, f"S={S} d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("S,d,causal,kl", [(1, 128, False, None), (1, 64, True, [31000, 7]),
+                                           (37, 128, True, [40000, 129]), (256, 64, False, [39999, 40000]),
+                                           (5, 64, False, [0, 300])])
+def test_splitkv_single_row_long_keys(S, d, causal, kl):
+    # one query row per head (the decode kernel): N_k = 40000 with a ragged tail,
+    # key lengths that end inside a tile, on a tile boundary, or at 0
+    B, H, Nq, Nk = 2, 3, 1, 40000
+    seed = 950 + S + d
+    q = normal_bf16((B, H, Nq, d), seed, 0)
+    k = normal_bf16((B, H, Nk, d), seed, 1)
+    v = normal_bf16((B, H, Nk, d), seed, 2)
+    scale = 1.0 / np.sqrt(d)
+    kl_arr = None if kl is None else np.array(kl, np.int32)
+    o, lse, guards = run_splitkv(q, k, v, scale, causal, kl_arr, S)
+    assert guards, "wrote outside O / LSE"
+    o_ref, lse_ref = oracle.attn_ref(q, k, v, scale, causal, kl_arr)
+    compare(o, lse, o_ref, lse_ref, f"S={S} d={d} causal={causal} kl={kl}")
+
+
 def test_splitkv_num_splits_uses_the_device_sm_count():
     import torch
     from io_aware_exact_24_b200 import fa_splitkv_num_splits
