@@ -41,6 +41,8 @@ NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ["io_aware_exact_24_b200/csrc/fa_fwd_kernel.cuh",
+                  "io_aware_exact_24_b200/csrc/fa_fwd_persist.cuh",
+                  "io_aware_exact_24_b200/csrc/fa_decode_kernel.cuh",
                   "io_aware_exact_24_b200/csrc/sm100_ptx.cuh",
                   "io_aware_exact_24_b200/csrc/exp2_poly.cuh",
                   "io_aware_exact_24_b200/csrc/fa_api.cu"]
