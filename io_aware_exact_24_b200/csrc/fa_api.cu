@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -50,6 +51,10 @@ constexpr unsigned kHeadGroupMinBlocks = 32;
 // Longest K/V walk (tiles of 128 keys) for which the dense forward uses persistent CTAs.
 constexpr int kPersistMaxTiles = 16;
 constexpr int kMaxDevices = 64;
+// fa_fwd_host pipelines its copies in chunks of heads: about this many chunks,
+// at most kHostChunksMax
+constexpr int kHostChunksTarget = 16;
+constexpr int kHostChunksMax = 64;
 // largest relative-position radius of a bias table (2^30: the table's
 // 2R+1 entries and every clamped index stay within int range)
 constexpr int kMaxBiasRadius = 1 << 30;
@@ -926,6 +931,35 @@ size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d, int has
     return host_layout(B, H, N_q, N_k, d, has_key_lens).total;
 }
 
+// Copy streams and events of fa_fwd_host, per device, created on first use.
+// Calls on one device are serialised (they are synchronous anyway).
+struct HostPipe {
+    std::once_flag once;
+    std::mutex mu;
+    cudaError_t status = cudaSuccess;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, last_out = nullptr;
+    cudaEvent_t in_done[kHostChunksMax] = {};
+    cudaEvent_t fwd_done[kHostChunksMax] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+HostPipe* host_pipe(int dev) {
+    HostPipe& hp = g_host_pipe[dev];
+    std::call_once(hp.once, [&] {
+        cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.last_out, cudaEventDisableTiming);
+        for (int i = 0; i < kHostChunksMax && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.fwd_done[i], cudaEventDisableTiming);
+        }
+        hp.status = e;
+    });
+    return &hp;
+}
+
 int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
                 int d, float scale, int causal, const int32_t* key_lens, void* workspace, size_t workspace_bytes,
                 fa_stream_t stream) {
@@ -935,26 +969,78 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse
     const HostLayout L = host_layout(B, H, N_q, N_k, d, key_lens != nullptr);
     if (workspace == nullptr || workspace_bytes < L.total) return FA_ERR_INVALID_ARG;
     if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    HostPipe* hp = host_pipe(dev);
+    if (hp->status != cudaSuccess) return cuda_fail("copy streams for fa_fwd_host", hp->status);
+    std::lock_guard<std::mutex> lock(hp->mu);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
-    const size_t bh = (size_t)B * H;
-    const size_t q_bytes = bh * N_q * d * 2, kv_bytes = bh * N_k * d * 2;
-    cudaError_t e = cudaMemcpyAsync(ws + L.q, q, q_bytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && kv_bytes > 0) e = cudaMemcpyAsync(ws + L.k, k, kv_bytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && kv_bytes > 0) e = cudaMemcpyAsync(ws + L.v, v, kv_bytes, cudaMemcpyHostToDevice, s);
+    const size_t q_head = (size_t)N_q * d * 2, kv_head = (size_t)N_k * d * 2;
+    // Chunks of about 1/kHostChunksTarget of the (b, h) pairs: runs of heads inside
+    // one batch entry, or of whole batch entries when a batch entry is smaller than
+    // that.  The copies of chunk c+1 and the read-back of chunk c-1 overlap the
+    // forward of chunk c (H2D and D2H on their own streams and copy engines), so the
+    // call costs about the longer of the two transfers instead of their sum.
+    const long long total = (long long)B * H;
+    const long long want = (total + kHostChunksTarget - 1) / kHostChunksTarget;   // pairs per chunk
+    const bool by_heads = want <= H;
+    const int per = by_heads ? (int)std::max(1LL, want) : H;                      // heads per chunk
+    const int per_b = by_heads ? (H + per - 1) / per : 1;                         // chunks per batch entry
+    const int bc = by_heads ? 1 : (int)((want + H - 1) / H);                      // batch entries per chunk
+    const int n_chunks = by_heads ? B * per_b : (B + bc - 1) / bc;
+    // at most 2 * kHostChunksTarget chunks (heads: B <= target; batches: <= target)
+    if (n_chunks > kHostChunksMax) return FA_ERR_UNSUPPORTED;
+    // the workspace may still be in use by earlier work on `stream`
+    e = cudaEventRecord(hp->start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->start, 0);
     const int32_t* kl_dev = nullptr;
     if (e == cudaSuccess && key_lens != nullptr) {
-        e = cudaMemcpyAsync(ws + L.kl, key_lens, (size_t)B * 4, cudaMemcpyHostToDevice, s);
+        e = cudaMemcpyAsync(ws + L.kl, key_lens, (size_t)B * 4, cudaMemcpyHostToDevice, hp->h2d);
         kl_dev = reinterpret_cast<const int32_t*>(ws + L.kl);
     }
-    if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (host to device)", e);
-    st = fa_fwd(ws + L.q, N_k > 0 ? ws + L.k : nullptr, N_k > 0 ? ws + L.v : nullptr, ws + L.o,
-                reinterpret_cast<float*>(ws + L.lse), B, H, N_q, N_k, d, scale, causal, kl_dev, stream);
-    if (st != FA_OK) return st;
-    e = cudaMemcpyAsync(o, ws + L.o, q_bytes, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(lse, ws + L.lse, bh * N_q * 4, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (device to host)", e);
-    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail("fa_fwd_host setup", e);
+    for (int c = 0; c < n_chunks; ++c) {
+        const int b = by_heads ? c / per_b : c * bc;
+        const int nb = by_heads ? 1 : std::min(bc, B - b);     // batch entries of the chunk
+        const int h0 = by_heads ? (c % per_b) * per : 0;
+        const int hc = by_heads ? std::min(per, H - h0) : H;   // heads per batch entry
+        const size_t row0 = (size_t)b * H + h0;                 // first (b, h) pair of the chunk
+        const size_t rows = (size_t)nb * hc;                    // (b, h) pairs of the chunk
+        e = cudaMemcpyAsync(ws + L.q + row0 * q_head, static_cast<const char*>(q) + row0 * q_head, rows * q_head,
+                            cudaMemcpyHostToDevice, hp->h2d);
+        if (e == cudaSuccess && kv_head > 0)
+            e = cudaMemcpyAsync(ws + L.k + row0 * kv_head, static_cast<const char*>(k) + row0 * kv_head,
+                                rows * kv_head, cudaMemcpyHostToDevice, hp->h2d);
+        if (e == cudaSuccess && kv_head > 0)
+            e = cudaMemcpyAsync(ws + L.v + row0 * kv_head, static_cast<const char*>(v) + row0 * kv_head,
+                                rows * kv_head, cudaMemcpyHostToDevice, hp->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(hp->in_done[c], hp->h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->in_done[c], 0);
+        if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (host to device)", e);
+        // the chunk as a problem of its own: nb batch entries of hc heads
+        st = fa_fwd(ws + L.q + row0 * q_head, N_k > 0 ? ws + L.k + row0 * kv_head : nullptr,
+                    N_k > 0 ? ws + L.v + row0 * kv_head : nullptr, ws + L.o + row0 * q_head,
+                    reinterpret_cast<float*>(ws + L.lse) + row0 * N_q, nb, hc, N_q, N_k, d, scale, causal,
+                    kl_dev != nullptr ? kl_dev + b : nullptr, stream);
+        if (st != FA_OK) return st;
+        e = cudaEventRecord(hp->fwd_done[c], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->fwd_done[c], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<char*>(o) + row0 * q_head, ws + L.o + row0 * q_head, rows * q_head,
+                                cudaMemcpyDeviceToHost, hp->d2h);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(lse + row0 * N_q, ws + L.lse + row0 * N_q * 4, rows * N_q * 4,
+                                cudaMemcpyDeviceToHost, hp->d2h);
+        if (e != cudaSuccess) return cuda_fail("cudaMemcpyAsync (device to host)", e);
+    }
+    // `stream` is complete only after the last read-back
+    e = cudaEventRecord(hp->last_out, hp->d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->last_out, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     return e == cudaSuccess ? FA_OK : cuda_fail("cudaStreamSynchronize", e);
 }
 

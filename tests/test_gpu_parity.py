@@ -179,15 +179,23 @@ def test_zero_query_gives_mean_of_values():
                                rtol=0, atol=1e-3)
 
 
-def test_host_entry_matches_device_entry():
+@pytest.mark.parametrize("shape", [(2, 3, 333, 257, 128, True), (2, 20, 300, 300, 64, False),
+                                   (40, 2, 200, 150, 64, True)],
+                         ids=["heads-6-chunks", "heads-20-per-batch", "whole-batches"])
+def test_host_entry_matches_device_entry(shape):
+    # the host entry copies and computes in chunks of heads (or of whole batch
+    # entries when a batch entry is small); every chunk is its own launch, and the
+    # result must be the device entry's, bit for bit
     import torch
     from io_aware_exact_24_b200 import fa_fwd_host, fa_fwd_host_workspace_size
-    B, H, Nq, Nk, d = 2, 3, 333, 257, 128
-    q, k, v = _rand(B, H, Nq, Nk, d, 81)
-    kl = np.array([200, 257], np.int32)
+    B, H, Nq, Nk, d, with_kl = shape
+    q, k, v = _rand(B, H, Nq, Nk, d, 81 + B + H)
+    kl = np.array([(Nk * (i + 1)) // B for i in range(B)], np.int32) if with_kl else None
+    if with_kl:
+        kl[0] = max(1, Nk - 57)
     dev = {}
     run_fa(q, k, v, 0.088, True, kl, out=dev)
-    ws_bytes = fa_fwd_host_workspace_size(B, H, Nq, Nk, d, True)
+    ws_bytes = fa_fwd_host_workspace_size(B, H, Nq, Nk, d, with_kl)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     o = np.empty((B, H, Nq, d), np.uint16)
     lse = np.empty((B, H, Nq), np.float32)
