@@ -202,14 +202,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t tmem = *tmem_holder;
 
     // The next block of a mailbox reader (k = blocks taken so far): wait for the
-    // scheduler's answer for block k+1, hand the slot back, and return false
-    // when there is none (or the wait ran out).  One lane waits, reads and
+    // scheduler's answer for block k+1 and hand the slot back; returns 1 with the
+    // item, 0 when the scheduler has none, -1 when the wait ran out.  One lane waits, reads and
     // arrives; with whole_warp the answer is broadcast to the other lanes, so
     // that the warp takes the same branch.  The single-lane roles (producer
     // and issuer lanes) call it with whole_warp = false from their own lane.
-    auto next_item = [&](int k, FwdItem& it, bool whole_warp) -> bool {
+    auto next_item = [&](int k, FwdItem& it, bool whole_warp) -> int {
         const int s = k & 1;
-        int m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int m[8] = {0, 0, 0, 0, 0, 0, 0, -1};   // m[7]: 1 item, 0 none, -1 the wait ran out
         if (!whole_warp || lane == 0) {
             if (wait_bounded(bar_item_ready(s), (uint32_t)((k >> 1) & 1), abort_flag, p.wait_limit)) {
                 const volatile int* mv = mailbox + 8 * s;
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) m[i] = __shfl_sync(0xffffffffu, m[i], 0);
         }
-        if (m[7] == 0) return false;
+        if (m[7] <= 0) return m[7];
         it.h = m[0];
         it.b = m[1];
         it.m0 = m[2];
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         it.off = m[4];
         it.t0 = m[5];
         it.n_kv = m[6];
-        return true;
+        return 1;
     };
 
     if (warp >= kProducerWarp) {
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     mbar_arrive(bar_item_ready(s));   // release: the mailbox writes above are visible
                     if (!got) break;
                 } else {
-                    if (!next_item(k, it, false)) break;
+                    if (next_item(k, it, false) <= 0) break;
                 }
             }
             // wind-down: every copy this producer issued that may still be in
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                     ++nq;
                 }
-                if (!next_item(k, it, false)) break;
+                if (next_item(k, it, false) <= 0) break;
             }
             // both issuers: every product issued has landed before TMEM is freed
             umma_commit(bar_fin);
@@ -570,7 +570,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             }
             epi[g * kBlockM + r] = m_seen;
             epi[(2 + g) * kBlockM + r] = lu;
-            good = !named_bar_or(kBarQuadBase + qd, 64, !good);
+            // The next block's item, read before the quadrant's barrier: both warps
+            // read the same mailbox slot, and a read whose wait ran out counts as a
+            // failure of this block, so the two warps leave together here (a warp
+            // left alone at the next block's barrier would wait without a limit).
+            const int nxt = next_item(k, it, true);
+            good = !named_bar_or(kBarQuadBase + qd, 64, !(good && nxt >= 0));
             const float m0w = epi[r], m1w = epi[kBlockM + r];
             const float m_fin = fmaxf(m0w, m1w);
             const float f0 = (m0w == m_fin) ? 1.f : ex2_approx(m0w - m_fin);
@@ -628,7 +633,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 mr_other += (g == 0) ? (n_kv - 1) / 2 : n_kv / 2;
                 ++nq;
             }
-            if (!next_item(k, it, true)) break;
+            if (nxt <= 0) break;   // the same answer in both warps (same mailbox slot)
         }
         tc_fence_before();
     }

@@ -42,6 +42,7 @@ class Persist(Fwd):
         self.item_ready = [b(f"item_ready{s}", 1) for s in range(2)]
         self.item_used = [b(f"item_used{s}", 11) for s in range(2)]
         self.quad = [b(f"quad{q}", 2) for q in range(4)]   # the epilogue's named barrier
+        self.go = {}                     # (q, block) -> the two warps' next-item answers
         self.mail = [None, None]
         self.q_block = None              # block whose Q is in the Q buffer
         self.qk_block_done = {}          # block -> QK^T products finished
@@ -251,8 +252,16 @@ def softmax(m, q, g):
             if m.pv_block.get(k, 0) != n or m.o_block != k:
                 m.errors.append(f"epilogue of block {k} after {m.pv_block.get(k, 0)} of {n} PVs (O of {m.o_block})")
         m.epi[(k & 1, q, g)] = k
+        # the next block's item is read before the quadrant's barrier, so the two warps
+        # take the decision to go on together (the kernel folds a read that ran out
+        # into the barrier's failure flag)
+        nxt = yield from take_next(m, k)
+        m.go.setdefault((q, k), []).append(nxt)
         m.quad[q].arrive()
         yield wait(m.quad[q], n_epi)
+        answers = m.go[(q, k)]
+        if len(answers) != 2 or answers[0] != answers[1]:
+            m.errors.append(f"q{q}: the warps of a quadrant disagree after block {k}: {answers}")
         n_epi += 1
         yield ("delay", m.lat(1, 300))
         if m.epi.get((k & 1, q, g ^ 1)) != k:
@@ -267,7 +276,6 @@ def softmax(m, q, g):
             sf_own += (n + 1) // 2 if g == 0 else n // 2
             mr_other += (n - 1) // 2 if g == 0 else n // 2
             nq += 1
-        nxt = yield from take_next(m, k)
         if nxt is None:
             return
         k = nxt

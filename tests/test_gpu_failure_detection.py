@@ -34,18 +34,21 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert fa_get_device_status() == FA_OK
 
 
-@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
-def test_forward_wait_limit_runs_out_and_context_survives(d, causal):
+@pytest.mark.parametrize("d,causal,B,H,N", [(64, False, 2, 4, 1000), (128, True, 2, 4, 1000),
+                                           (64, True, 4, 40, 512)],
+                         ids=["d64", "d128-causal", "d64-persistent"])
+def test_forward_wait_limit_runs_out_and_context_survives(d, causal, B, H, N):
     # The forward kernel itself with a wait limit of a few cycles: some pipeline
     # wait runs out, every role of that CTA stops after its own copies and MMAs
     # have landed, and the call reports FA_ERR_DEVICE_TIMEOUT.  The context must
     # stay usable: a normal call afterwards passes parity and leaves the status clean.
+    # The last case has 640 short blocks, so it runs the persistent CTA (the
+    # scheduler, the mailbox and the block-to-block hand-offs wind down too).
     import torch
     from io_aware_exact_24_b200 import (FA_ERR_DEVICE_TIMEOUT, FA_OK, fa_get_device_status,
                                         fa_selftest_fwd_timeout)
     from fa_testutil import to_device_bf16
     assert fa_get_device_status() == FA_OK
-    B, H, N = 2, 4, 1000
     q = normal_bf16((B, H, N, d), 6 + d, 0)
     k = normal_bf16((B, H, N, d), 6 + d, 1)
     v = normal_bf16((B, H, N, d), 6 + d, 2)
