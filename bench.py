@@ -717,6 +717,13 @@ def main():
                             "frac_of_nominal_2250": wn.flop / (ms_n / 1000.0) / 1e12 / NOMINAL_BF16_TFLOPS,
                             "algorithmic_gbs": wn.algorithmic_bytes / (ms_n / 1000.0) / 1e9,
                             "l2": "flushed between launches"}
+            if xn["key_lens"] is not None:
+                # padded batches: also the FLOPs of the keys each sequence has
+                # (4*H*d*N_q*sum_b key_len_b, causal halved), beside the formula's
+                kl = np.clip(np.asarray(xn["key_lens"], np.int64), 0, wn.Nk)
+                eff = 4.0 * wn.H * wn.d * wn.Nq * float(kl.sum()) * (0.5 if wn.causal else 1.0)
+                per_wl[name]["effective"] = {"flop": eff, "tflops": eff / (ms_n / 1000.0) / 1e12,
+                                             "flop_formula": "4*H*d*N_q*sum_b key_len_b"}
             if wn.algorithmic_bytes < (126 << 20):
                 # inputs that fit in L2: also back-to-back launches on a warm L2
                 ms_w, per_w, _ = time_device(wn, xn, args.steps, args.warmup, device, 0, 1,
