@@ -302,8 +302,9 @@ FA_API int fa_fwd_host(const void *q, const void *k, const void *v, void *o, flo
  * counts its arrival for its query block; the last of the block's CTAs to
  * arrive merges the ranges of the block's rows: with M = max_s LSE_s and
  * w_s = exp(LSE_s - M), O = sum_s w_s O_s / sum_s w_s and LSE = M + ln sum_s w_s
- * (a row with no visible key in any range: O = 0, LSE = -inf).  One memset of
- * the arrival counters and one kernel launch per call.  This is the
+ * (a row with no visible key in any range: O = 0, LSE = -inf).  One kernel
+ * launch per call: the arrival words carry a ticket drawn for each call, so
+ * they need no reset between calls.  This is the
  * decode / FlashDecoding case "FlashAttention：把注意力从公式写成数据流"
  * (section "端侧与专用加速器") and "[2205.14135] FlashAttention: Fast and
  * Memory-Efficient Exact Attention with IO-Awareness" point to, merged with the
@@ -325,7 +326,7 @@ FA_API int fa_splitkv_num_splits(int B, int H, int N_q, int N_k);
 /*
  * fa_fwd_splitkv_workspace_size -- bytes of device workspace fa_fwd_splitkv
  * needs: num_splits*B*H*N_q*d fp32 partial outputs, num_splits*B*H*N_q fp32
- * partial LSEs and ceil(N_q/128)*B*H int32 arrival counters, each part 256-byte
+ * partial LSEs and ceil(N_q/128)*B*H 64-bit arrival words, each part 256-byte
  * aligned.  Returns 0 for invalid sizes or num_splits outside [1, 256].
  */
 FA_API size_t fa_fwd_splitkv_workspace_size(int B, int H, int N_q, int d, int num_splits);

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -241,37 +243,24 @@ bool encode_dq_acc(CUtensorMap* map, float* ptr, int BH, int N, int d) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-__global__ void zero_ints_kernel(int* p, int n) {
-    fa::pdl_launch_dependents();   // the split kernel touches the counters only after waiting
-    const int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
-    if (i < n) p[i] = 0;
+// A 48-bit ticket for each split-KV call: the arrival words in the workspace
+// carry it, so they need no reset between calls (see split_arrive_last).  The
+// sequence starts at a value taken from the clock, so a workspace left by
+// another process is unlikely to hold a current ticket.
+unsigned long long next_split_ticket() {
+    static std::atomic<unsigned long long> seq{(unsigned long long)std::chrono::steady_clock::now()
+                                                   .time_since_epoch()
+                                                   .count() *
+                                               0x9E3779B97F4A7C15ull};
+    return (seq.fetch_add(1, std::memory_order_relaxed) + 1) & ((1ull << 48) - 1);
 }
 
-// Launch a kernel that may start while the previous kernel of the stream (the
-// counters' zeroing) still runs; it waits for that kernel before its first use
-// of the counters (programmatic dependent launch).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                             Args&&... args) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
-// Split-KV: partial results and per-block arrival counters in the workspace.
+// Split-KV: partial results and per-block arrival words in the workspace.
 struct SplitParts {
     int num_splits;   // 0: plain forward
     float* o_part;
     float* lse_part;
-    int* counter;     // [B, H, query blocks]
+    unsigned long long* counter;   // arrival words [B, H, query blocks]
 };
 
 // Packed [T, H, d] bf16 viewed as (d, H, T, 1), box 64 x 1 x 128 x 1: the same
@@ -366,6 +355,7 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.o_part = sp.o_part;
     p.lse_part = sp.lse_part;
     p.split_counter = sp.counter;
+    p.split_ticket = sp.num_splits > 0 ? next_split_ticket() : 0;
     p.o_out = reinterpret_cast<__nv_bfloat16*>(o);
     p.o_scale = o_scale;
     const int rows_per_cta = fa::kBlockM;
@@ -424,25 +414,19 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
         const cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch", e);
     }
-    // the arrival counters start at zero (the workspace has no required contents);
-    // a kernel on the same engine as the next launch, not a memset operation,
-    // which measured about 15 us of stream time on decode-sized calls
-    const int n_counters = (int)((size_t)num_m * H * B);
-    zero_ints_kernel<<<(unsigned)((n_counters + 255) / 256), 256, 0, stream>>>(sp.counter, n_counters);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail("kernel launch (split-KV counters)", e);
+    // the arrival words need no reset: each call's arrivals carry its own ticket
+    cudaError_t e;
     if (N_q == 1) {
         // one query row: matrix-vector products, streamed on the CUDA cores
         dim3 grid((unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
-        e = launch_dependent(fa::fa_decode_splitkv_kernel<D>, grid, dim3(fa::kDecThreads), fa::DecCfg<D>::kSmemBytes,
-                             stream, tk, tv, reinterpret_cast<const __nv_bfloat16*>(q), p);
-        if (e == cudaSuccess) e = cudaGetLastError();
+        fa::fa_decode_splitkv_kernel<D><<<grid, fa::kDecThreads, fa::DecCfg<D>::kSmemBytes, stream>>>(
+            tk, tv, reinterpret_cast<const __nv_bfloat16*>(q), p);
+        e = cudaGetLastError();
         return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (decode)", e);
     }
     dim3 grid(num_m * (unsigned)sp.num_splits, (unsigned)H, (unsigned)B);
-    e = launch_dependent(fa::fa_fwd_sm100_kernel<D, true>, grid, dim3(fa::kNumThreads), fa::Cfg<D>::kSmemBytes, stream,
-                         tq, tk, tv, to, p);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    fa::fa_fwd_sm100_kernel<D, true><<<grid, fa::kNumThreads, fa::Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    e = cudaGetLastError();
     return e == cudaSuccess ? FA_OK : cuda_fail("kernel launch (split-KV)", e);
     }
 }
@@ -461,8 +445,8 @@ int current_num_sms() {
     return n;
 }
 
-// Workspace of the split-KV forward: O partials, LSE partials, then one int32
-// arrival counter per (query block, head, batch), each 256-byte aligned.
+// Workspace of the split-KV forward: O partials, LSE partials, then one
+// 64-bit arrival word per (query block, head, batch), each part 256-byte aligned.
 struct SplitLayout {
     size_t o_part, lse_part, counter, total;
 };
@@ -473,7 +457,7 @@ SplitLayout split_layout(int B, int H, int N_q, int d, int num_splits) {
     L.o_part = 0;
     L.lse_part = (rows * d * 4 + 255) / 256 * 256;
     L.counter = L.lse_part + (rows * 4 + 255) / 256 * 256;
-    L.total = L.counter + (blocks * 4 + 255) / 256 * 256;
+    L.total = L.counter + (blocks * 8 + 255) / 256 * 256;
     return L;
 }
 
@@ -663,7 +647,7 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part),
-                        reinterpret_cast<int*>(ws + L.counter)};
+                        reinterpret_cast<unsigned long long*>(ws + L.counter)};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }
@@ -731,13 +715,12 @@ int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o,
     void* scratch = nullptr;
     st = scratch_address(dev, &scratch);
     if (st != FA_OK) return st;
-    // Every partial the merge reads is written first, and the arrival counters
-    // are zeroed on the stream before the kernel, so nothing in the scratch has
-    // to start at zero.
+    // Every partial the merge reads is written first, and the arrival words carry
+    // each call's own ticket, so nothing in the scratch has to start at zero.
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(scratch);
     const SplitParts sp{num_splits, reinterpret_cast<float*>(ws + L.o_part), reinterpret_cast<float*>(ws + L.lse_part),
-                        reinterpret_cast<int*>(ws + L.counter)};
+                        reinterpret_cast<unsigned long long*>(ws + L.counter)};
     if (d == 64) return launch<64>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
     return launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, key_lens, s, sp);
 }

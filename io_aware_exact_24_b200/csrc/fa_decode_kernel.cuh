@@ -276,29 +276,41 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (lane == 0) p.lse_part[(size_t)split * rows_total + rg] = lse;
     __threadfence();   // the partial is visible before the arrival below
     __syncwarp();
-    // the counters were zeroed by the kernel launched just before this one, which
-    // this kernel may overlap (programmatic dependent launch)
-    pdl_wait_primary();
-    if (lane == 0) *merge_flag = (atomicAdd(p.split_counter + rg, 1) == n_split - 1) ? 1 : 0;
+    if (lane == 0) *merge_flag = split_arrive_last(p.split_counter + rg, p.split_ticket, n_split) ? 1 : 0;
     __syncwarp();
     if (!*merge_flag) return;
-    // the last range of this row to arrive merges all of them (running-max rule)
+    // the last range of this row to arrive merges all of them (running-max rule):
+    // the ranges' LSEs a range per lane, their partial O rows with eight loads in
+    // flight per lane, so the merge is not a chain of dependent L2 round trips
     __threadfence();
     float ml = -INFINITY;
-    for (int sp = 0; sp < n_split; ++sp) ml = fmaxf(ml, __ldcg(p.lse_part + (size_t)sp * rows_total + rg));
+    for (int s0 = 0; s0 < n_split; s0 += 32) {
+        const int sp = s0 + lane;
+        if (sp < n_split) ml = fmaxf(ml, __ldcg(p.lse_part + (size_t)sp * rows_total + rg));
+    }
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) ml = fmaxf(ml, __shfl_xor_sync(0xffffffffu, ml, sh));
     float wsum = 0.f;
     float out[kOw];
 #pragma unroll
     for (int e = 0; e < kOw; ++e) out[e] = 0.f;
     if (ml != -INFINITY) {
-        for (int sp = 0; sp < n_split; ++sp) {
-            const float ls = __ldcg(p.lse_part + (size_t)sp * rows_total + rg);
+        for (int s0 = 0; s0 < n_split; s0 += 32) {
+            const int sp = s0 + lane;
+            const float ls = (sp < n_split) ? __ldcg(p.lse_part + (size_t)sp * rows_total + rg) : -INFINITY;
             const float w = (ls == -INFINITY) ? 0.f : expf(ls - ml);
-            const float* src = p.o_part + ((size_t)sp * rows_total + rg) * D + lane * kOw;
-#pragma unroll
-            for (int e = 0; e < kOw; ++e) out[e] = fmaf(w, __ldcg(src + e), out[e]);
             wsum += w;
+            const int cnt = min(32, n_split - s0);
+#pragma unroll 8
+            for (int t = 0; t < cnt; ++t) {
+                const float wt = __shfl_sync(0xffffffffu, w, t);
+                const float* src = p.o_part + ((size_t)(s0 + t) * rows_total + rg) * D + lane * kOw;
+#pragma unroll
+                for (int e = 0; e < kOw; ++e) out[e] = fmaf(wt, __ldcg(src + e), out[e]);
+            }
         }
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, sh);
     }
     const float winv = (wsum > 0.f) ? 1.f / wsum : 0.f;
     __nv_bfloat16* dst = p.o_out + rg * D + lane * kOw;

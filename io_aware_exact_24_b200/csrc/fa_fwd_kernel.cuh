@@ -109,9 +109,11 @@ struct FwdParams {
     int num_splits;
     float* o_part;              // [num_splits, B, H, Nq, D] fp32, O of the range / its own l
     float* lse_part;            // [num_splits, B, H, Nq] fp32, LSE of the range (-inf if empty)
-    // arrivals per (query block, h, b), [B, H, num query blocks], zero at launch: the
-    // last CTA of a query block to finish merges its ranges into o_out / lse
-    int* split_counter;
+    // arrival words per (query block, h, b), [B, H, num query blocks], any initial
+    // contents: (ticket << 16) | arrivals of the call whose ticket is split_ticket;
+    // the last CTA of a query block to arrive merges its ranges into o_out / lse
+    unsigned long long* split_counter;
+    unsigned long long split_ticket;   // 48 bits, different for every call
     __nv_bfloat16* o_out;       // final O [B,H,Nq,D] of the split-KV mode
     // dense single-pass mode: > 1 reorders the CTAs' work (see the kernel); 0 or 1 keeps
     // blockIdx = (query block, h, b)
@@ -338,6 +340,22 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
     return c < kl ? (int)c : kl;
 }
 
+// Counts one arrival of this call's CTAs of a query block and tells whether it
+// was the last of n.  The word holds (ticket << 16) | count.  An arrival that
+// finds another ticket there (an earlier call, or whatever the workspace held)
+// tries once to claim the word with (ticket << 16) | 0: the first claim wins,
+// and every later claim fails because the word has changed, so it needs no
+// retry; then each arrival adds 1 (one atomic, no retry loop however many
+// ranges arrive at once).  Every add lands on a word that already carries this
+// call's ticket, so the words need no reset between calls; two calls share a
+// word only if their 48-bit tickets are equal.
+__device__ __forceinline__ bool split_arrive_last(unsigned long long* word, unsigned long long ticket, int n) {
+    const unsigned long long cur = atomicAdd(word, 0ull);
+    if ((cur >> 16) != ticket) atomicCAS(word, cur, ticket << 16);
+    const unsigned long long old = atomicAdd(word, 1ull);
+    return (int)(old & 0xffffull) + 1 == n;
+}
+
 // Split-KV merge, run by the 256 softmax threads of a CTA once its partial
 // (O_s, LSE_s) is in global memory: the CTA counts its arrival for its query
 // block, and the last of the block's num_splits CTAs to arrive merges every
@@ -348,8 +366,8 @@ __device__ __forceinline__ int row_key_limit(int row, int kl, int off, int causa
 // row whose ranges are all empty (M = -inf) gets O = 0, LSE = -inf; an empty
 // range has LSE_s = -inf, so w_s = 0 and its O_s (zeros) adds nothing.  Work
 // items are (row, 4 columns), spread over the 256 threads, so a decode block
-// with one row still loads its ranges' partials in parallel.  The counters are
-// zeroed on the stream before every launch.
+// with one row still loads its ranges' partials in parallel.  The arrival
+// words need no reset (split_arrive_last).
 template <int D>
 __device__ __forceinline__ void split_merge(const FwdParams& p, uint8_t* flag_smem, int n_split, int num_m, int m_blk,
                                             int m0, int h, int b) {
@@ -358,9 +376,7 @@ __device__ __forceinline__ void split_merge(const FwdParams& p, uint8_t* flag_sm
     if (threadIdx.x == 0) {
         // every softmax thread fenced its own partial stores before the barrier
         // that preceded this arrival
-        pdl_wait_primary();   // the counters' zeroing kernel (it may still run: dependent launch)
-        const int old = atomicAdd(p.split_counter + grp, 1);
-        *flag = (old == n_split - 1) ? 1 : 0;
+        *flag = split_arrive_last(p.split_counter + grp, p.split_ticket, n_split) ? 1 : 0;
     }
     named_bar_sync(kBarSoftmaxAll, kSoftmaxWarps * 32);
     if (!*flag) return;

@@ -291,12 +291,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 // the compiler cannot move its first use above the wait.
 __device__ __forceinline__ void reg_after_wait(uint32_t& x) { asm volatile("" : "+r"(x)); }
 
-// Programmatic dependent launch: let the next kernel of the stream start its
-// prologue now (primary side), and wait until the preceding kernel has finished
-// and its writes are visible (dependent side; a no-op without the launch attribute).
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // 16-byte shared-memory load of four floats (address in the shared window).
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, float& a, float& b, float& c, float& d) {
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(a), "=f"(b), "=f"(c), "=f"(d) : "r"(addr));

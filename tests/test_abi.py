@@ -133,8 +133,8 @@ def test_splitkv_workspace_size_formula(lib):
         rows = S * B * H * Nq
         need = binding.fa_fwd_splitkv_workspace_size(B, H, Nq, d, S)
         o_bytes = -(-rows * d * 4 // 256) * 256
-        blocks = -(-Nq // 128) * B * H          # one int32 arrival counter per query block
-        assert need == o_bytes + -(-rows * 4 // 256) * 256 + -(-blocks * 4 // 256) * 256
+        blocks = -(-Nq // 128) * B * H          # one 64-bit arrival word per query block
+        assert need == o_bytes + -(-rows * 4 // 256) * 256 + -(-blocks * 8 // 256) * 256
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 96, 2) == 0
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 0) == 0
     assert binding.fa_fwd_splitkv_workspace_size(1, 1, 1, 64, 257) == 0
