@@ -81,8 +81,8 @@ struct BwdCfg {
     static constexpr int kRowOff = kDQ2Off + (D == 128 ? 2 * kSwizzleBoxBytes : 0);   // [2][lse2 x128 | D x128] fp32
     static constexpr int kBarOff = kRowOff + 2 * 256 * 4;
     // barriers: kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], s_full,
-    // p_full, dq_full, s_free, drain
-    static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesO + 5;
+    // p_full (pass 0), dq_full, s_free, drain, p_full (pass 1)
+    static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesO + 6;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar_o_empty = [&](int s) { return bar(1 + 2 * C::kStagesQ + C::kStagesO + s); };
     constexpr int kB0 = 1 + 2 * C::kStagesQ + 2 * C::kStagesO;
     const uint32_t bar_s_full = bar(kB0);
-    const uint32_t bar_p_full = bar(kB0 + 1);
+    // P^T / dS^T of one compute pass written (pass h: queries 32h.. and 64 + 32h..)
+    auto bar_p_full = [&](int half) { return bar(half == 0 ? kB0 + 1 : kB0 + 5); };
     const uint32_t bar_dq_full = bar(kB0 + 2);
     const uint32_t bar_s_free = bar(kB0 + 3);
     const uint32_t bar_drain = bar(kB0 + 4);
@@ -177,7 +178,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(bar_o_empty(s), 1);
         }
         mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, kBwdComputeWarps);    // one arrival per compute warp
+        mbar_init(bar_p_full(0), kBwdComputeWarps);   // one arrival per compute warp and half
+        mbar_init(bar_p_full(1), kBwdComputeWarps);
         mbar_init(bar_dq_full, 1);
         mbar_init(bar_s_free, kBwdComputeWarps);
         mbar_init(bar_drain, 1);
@@ -271,23 +273,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             smem_desc_sw128(do_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar_s_full);
-                ok = wait_bounded(bar_p_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
+                // dV and dK for the queries of each pass as soon as the compute warps
+                // have written that pass's P^T and dS^T: the first pass's products
+                // overlap the second pass's exponentials.  Pass h covers the query
+                // blocks 32cb.. with cb = h and 2 + h, i.e. kk = 2h, 2h+1, 2h+4, 2h+5;
+                // P^T of queries 16kk.. sits at column 32(kk/2) + 8(kk%2) (dS^T
+                // likewise from kColDP).
+#pragma unroll 1
+                for (int half = 0; half < 2 && ok; ++half) {
+                    ok = wait_bounded(bar_p_full(half), (uint32_t)(t & 1), abort_flag, p.wait_limit);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {   // dV += P^T dO: 16 queries per step
+                        const int kk = 4 * (k4 / 2) + 2 * half + (k4 % 2);
+                        umma_ts(tmem + C::kColDV, tmem + C::kColS + (uint32_t)(32 * (kk / 2) + 8 * (kk % 2)),
+                                smem_desc_sw128(do_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024),
+                                C::kIdescKV, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (half == 1) umma_commit(bar_o_empty(so));   // dO_i is no longer read
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {   // dK += dS^T Q
+                        const int kk = 4 * (k4 / 2) + 2 * half + (k4 % 2);
+                        umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(32 * (kk / 2) + 8 * (kk % 2)),
+                                smem_desc_sw128(q_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024),
+                                C::kIdescKV, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
                 if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk) {   // dV += P^T dO: 16 queries per step
-                    // P^T of queries 16kk.. at column 8kk (first 64 queries) or 8kk + 32
-                    umma_ts(tmem + C::kColDV, tmem + C::kColS + (uint32_t)(kk * 8 + 32 * (kk / 4)),
-                            smem_desc_sw128(do_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
-                            (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(bar_o_empty(so));   // dO_i is no longer read
-#pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk) {   // dK += dS^T Q
-                    umma_ts(tmem + C::kColDK, tmem + C::kColDP + (uint32_t)(kk * 8 + 32 * (kk / 4)),
-                            smem_desc_sw128(q_s + (uint32_t)(kk * 16 * 128), kSwizzleBoxBytes, 1024), C::kIdescKV,
-                            (t > 0 || kk > 0) ? 1u : 0u);
-                }
                 umma_commit(bar_q_empty(sq));   // Q_i is no longer read
 #pragma unroll
                 for (int kk = 0; kk < 128 / 16; ++kk) {   // dQ = dS K: 16 keys per step
@@ -347,7 +360,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
 #pragma unroll 1
-            for (int cb = 2 * g; cb < 2 * g + 2; ++cb) {   // queries 32cb .. 32cb+31
+            for (int pass = 0; pass < 2; ++pass) {
+                // queries 32cb .. 32cb+31: each warp stays inside its own 64 queries, so
+                // its dS^T goes only to box g, where it alone stages dQ
+                const int cb = 2 * g + pass;
                 uint32_t su[32], du[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32u * cb, su);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32u * cb, du);
@@ -406,11 +422,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     body(std::true_type{});
                 else
                     body(std::false_type{});
-                // P^T over S^T's columns 16cb + 32g.., dS^T over dP^T's: inside the 64
-                // columns this warp has read (the other warp of the quadrant reads
-                // the other 64), and after this warp read them
-                tmem_st16(tmem + lane_off + C::kColS + 16u * cb + 32u * g, pw);
-                tmem_st16(tmem + lane_off + C::kColDP + 16u * cb + 32u * g, dw);
+                // P^T over the first 16 of the 32 S^T columns this warp has just read
+                // (32cb..), dS^T likewise over dP^T's: no other warp reads them
+                tmem_st16(tmem + lane_off + C::kColS + 32u * cb, pw);
+                tmem_st16(tmem + lane_off + C::kColDP + 32u * cb, dw);
                 // dS^T row r into shared memory: box cb/2 holds queries 64(cb/2)..+63 as
                 // 128-byte rows, 16-byte chunk cc at swizzled position cc ^ (r % 8)
 #pragma unroll
@@ -422,12 +437,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                  "r"(dw[4 * t4 + 1]), "r"(dw[4 * t4 + 2]), "r"(dw[4 * t4 + 3])
                                  : "memory");
                 }
+                tmem_wait_st();
+                fence_proxy_async_smem();   // dS^T visible to the tensor core
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_p_full(pass));
             }
-            tmem_wait_st();
-            fence_proxy_async_smem();   // dS^T visible to the tensor core
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_p_full);
             // dQ_i (TMEM lane = query row i0 + r) into the fp32 accumulator
             good = wait_bounded(bar_dq_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);
             if (!__all_sync(0xffffffffu, good)) {

@@ -11,6 +11,13 @@ latencies are drawn for copies, MMAs and compute.  Checked for every schedule:
   * the data each role consumes is the data of its own tile (Q/dO slot contents,
     S/dP contents, the dS^T buffer and the dQ columns), so no buffer is overwritten
     while still in use.
+Geometry as in the kernel: warp w serves TMEM lane quadrant qd and query half g; the
+tile's 128 queries are four blocks cb of 32.  A warp computes its blocks cb = 2g + pass
+in two passes and hands each pass over on p_full[pass]; the issuer runs dV and dK of
+pass h (blocks h and 2 + h) while the next pass is computed.  dS^T of block cb goes to
+shared-memory box cb // 2, rows of quadrant qd -- the region where warp (qd, g = box)
+stages its dQ for the tensor reduce.  S/dP columns are tracked per (block, quadrant),
+shared-memory regions per (box, quadrant).
 This checks the protocol as designed; the kernel is checked by the GPU parity tests.
 """
 import random
@@ -33,6 +40,29 @@ class Barrier:
         return (self.completed & 1) != parity
 
 
+def fill(cols, v):
+    for half in cols:
+        half[:] = [v] * len(half)
+
+
+def holds(cols, v):
+    return all(x == v for half in cols for x in half)
+
+
+def kernel_cb(pass_, g):
+    """Query block a warp of query half g computes in pass pass_."""
+    return 2 * g + pass_
+
+
+def kernel_pass_blocks(h):
+    """Query blocks the issuer's dV / dK of pass h read (kk = 2h, 2h+1, 2h+4, 2h+5)."""
+    return (h, 2 + h)
+
+
+BLOCKS = [(cb, qd) for cb in range(4) for qd in range(4)]
+REGIONS = [(box, qd) for box in range(2) for qd in range(4)]
+
+
 class Sim:
     def __init__(self, n_t, stages, seed, warps=8, stages_o=None):
         self.rng = random.Random(seed)
@@ -47,19 +77,27 @@ class Sim:
         self.q_empty = [b(f"q_empty{s}", 1) for s in range(stages)]
         self.o_full = [b(f"o_full{s}", 1) for s in range(self.SO)]
         self.o_empty = [b(f"o_empty{s}", 1) for s in range(self.SO)]
-        self.s_full, self.p_full = b("s_full", 1), b("p_full", warps)
+        self.s_full = b("s_full", 1)
+        self.p_full = [b(f"p_full{h}", warps) for h in range(2)]
         self.dq_full, self.s_free = b("dq_full", 1), b("s_free", warps)
         self.drain = b("drain", 1)
         # buffer contents: which tile's data they hold
         self.slot = [None] * stages           # Q slot -> tile
         self.oslot = [None] * self.SO         # dO slot -> tile
-        self.s_cols = None                    # S^T / P^T / dQ columns: ("S", t) / ("dQ", t)
-        self.dp_cols = None                   # dP^T / dS^T columns
-        self.ds_smem = None                   # dS^T in shared memory
-        self.stage = [None] * warps           # each warp's part of that buffer: ("dS", t) / ("dQ", t)
-        self.reading = [False] * warps        # a tensor reduce is still reading the warp's dQ staging
+        # per (block, quadrant): S^T / P^T / dQ columns ("S", t) / ("P", t) / ("dQ", t)
+        # and dP^T / dS^T columns ("dP", t) / ("dS", t)
+        self.s_cols = {k: None for k in BLOCKS}
+        self.dp_cols = {k: None for k in BLOCKS}
+        # per (box, quadrant) of the dS^T buffer: ("dS", t) / ("dQ", t), and whether a
+        # tensor reduce is still reading the dQ staged there
+        self.region = {k: None for k in REGIONS}
+        self.reading = {k: False for k in REGIONS}
         self.tc_free_at = 0                   # tensor core busy until
         self.errors = []
+
+    def fill_s(self, v):
+        for k in BLOCKS:
+            self.s_cols[k] = v
 
     def at(self, dt, fn):
         self.seq += 1
@@ -150,7 +188,7 @@ def producer(sim):
         yield ("delay", 1)
 
 
-def issuer(sim):
+def issuer(sim, pass_blocks=kernel_pass_blocks):
     yield wait(sim.kv, 0)
     for t in range(sim.n_t):
         s = t % sim.S
@@ -161,7 +199,7 @@ def issuer(sim):
         def mma1(t=t, s=s):
             if sim.slot[s] != t:
                 sim.errors.append(f"S of tile {t} read Q slot holding {sim.slot[s]}")
-            sim.s_cols = ("S", t)
+            sim.fill_s(("S", t))
         sim.mma(sim.lat(50, 150), mma1)
         so = t % sim.SO
         yield wait(sim.o_full[so], t // sim.SO)
@@ -169,67 +207,80 @@ def issuer(sim):
         def mma2(t=t, so=so):
             if sim.oslot[so] != t:
                 sim.errors.append(f"dP of tile {t} read dO slot holding {sim.oslot[so]}")
-            sim.dp_cols = ("dP", t)
+            for k in BLOCKS:
+                sim.dp_cols[k] = ("dP", t)
         sim.mma(sim.lat(50, 150), mma2)
         sim.commit(sim.s_full)
-        yield wait(sim.p_full, t)
+        for h in range(2):
+            yield wait(sim.p_full[h], t)
+            keys = [(cb, qd) for cb in pass_blocks(h) for qd in range(4)]
 
-        def mma3(t=t, so=so):
-            if sim.oslot[so] != t or sim.s_cols != ("P", t):
-                sim.errors.append(f"dV of tile {t} read dO {sim.oslot[so]}, {sim.s_cols}")
-        sim.mma(sim.lat(50, 150), mma3)
-        sim.commit(sim.o_empty[so])
+            def mma3(t=t, so=so, keys=keys):
+                if sim.oslot[so] != t or any(sim.s_cols[k] != ("P", t) for k in keys):
+                    sim.errors.append(f"dV of tile {t} read dO {sim.oslot[so]}, P^T {[sim.s_cols[k] for k in keys]}")
+            sim.mma(sim.lat(25, 75), mma3)
+            if h == 1:
+                sim.commit(sim.o_empty[so])
 
-        def mma4(t=t, s=s):
-            if sim.slot[s] != t or sim.dp_cols != ("dS", t):
-                sim.errors.append(f"dK of tile {t} read Q {sim.slot[s]}, {sim.dp_cols}")
-        sim.mma(sim.lat(50, 150), mma4)
+            def mma4(t=t, s=s, keys=keys):
+                if sim.slot[s] != t or any(sim.dp_cols[k] != ("dS", t) for k in keys):
+                    sim.errors.append(f"dK of tile {t} read Q {sim.slot[s]}, dS^T {[sim.dp_cols[k] for k in keys]}")
+            sim.mma(sim.lat(25, 75), mma4)
         sim.commit(sim.q_empty[s])
 
         def mma5(t=t):
-            if sim.ds_smem != t or any(st != ("dS", t) for st in sim.stage):
-                sim.errors.append(f"dQ of tile {t} read dS^T of {sim.ds_smem} / {sim.stage}")
-            sim.s_cols = ("dQ", t)
+            if any(sim.region[k] != ("dS", t) for k in REGIONS):
+                sim.errors.append(f"dQ of tile {t} read dS^T {sim.region}")
+            sim.fill_s(("dQ", t))
         sim.mma(sim.lat(50, 200), mma5)
         sim.commit(sim.dq_full)
         yield ("delay", 1)
     sim.commit(sim.drain)
 
 
-def compute_warp(sim, w, rows_barrier):
+def compute_warp(sim, w, rows_barrier, cb_of=kernel_cb):
+    qd, g = w % 4, w // 4
+    own = (g, qd)                       # where this warp stages dQ
     for t in range(sim.n_t):
         yield from rows_barrier(t)
         yield wait(sim.s_full, t)
-        if sim.s_cols not in (("S", t), ("P", t)) or sim.dp_cols not in (("dP", t), ("dS", t)):
-            sim.errors.append(f"warp {w} tile {t} read {sim.s_cols} {sim.dp_cols}")
-        yield ("delay", sim.lat(100, 800))
-        # the columns must still hold this tile's S / dP (or the other warps' P / dS)
-        # when the reads end
-        if sim.s_cols not in (("S", t), ("P", t)) or sim.dp_cols not in (("dP", t), ("dS", t)):
-            sim.errors.append(f"warp {w} tile {t}: S/dP overwritten during the read")
-        # dS^T goes where this warp staged the previous tile's dQ: its reduce must be done reading
-        while sim.reading[w]:
+        # the warp waits for its own dQ reduce to finish reading before any dS^T store
+        while sim.reading[own]:
             yield ("delay", 10)
-        sim.stage[w] = ("dS", t)
-        sim.s_cols, sim.dp_cols, sim.ds_smem = ("P", t), ("dS", t), t
-        sim.p_full.arrive()
+        for pass_ in range(2):
+            cb = cb_of(pass_, g)
+            blk, reg = (cb, qd), (cb // 2, qd)
+
+            def ok():
+                return sim.s_cols[blk] == ("S", t) and sim.dp_cols[blk] == ("dP", t)
+            if not ok():
+                sim.errors.append(f"warp {w} tile {t} block {cb} read {sim.s_cols[blk]} {sim.dp_cols[blk]}")
+            yield ("delay", sim.lat(50, 400))
+            # the block's columns must still hold this tile's S / dP when the reads end
+            if not ok():
+                sim.errors.append(f"warp {w} tile {t} block {cb}: S/dP overwritten during the read")
+            sim.s_cols[blk], sim.dp_cols[blk] = ("P", t), ("dS", t)
+            if sim.reading[reg]:
+                sim.errors.append(f"warp {w} tile {t}: dS^T written over dQ staging {reg} under a reduce")
+            sim.region[reg] = ("dS", t)
+            sim.p_full[pass_].arrive()
         yield wait(sim.dq_full, t)
-        if sim.s_cols != ("dQ", t):
+        if any(sim.s_cols[k] != ("dQ", t) for k in BLOCKS):
             sim.errors.append(f"warp {w} tile {t} read dQ from {sim.s_cols}")
         yield ("delay", sim.lat(50, 500))
-        if sim.s_cols != ("dQ", t):
+        if any(sim.s_cols[k] != ("dQ", t) for k in BLOCKS):
             sim.errors.append(f"warp {w} tile {t}: dQ overwritten during the read")
         sim.s_free.arrive()
-        # dQ staged in this warp's part of the dS^T buffer (the dQ product, its last
+        # dQ staged in this warp's region of the dS^T buffer (the dQ product, its last
         # reader, is done), then a tensor reduce reads it asynchronously
         yield ("delay", sim.lat(20, 200))
-        sim.stage[w] = ("dQ", t)
-        sim.reading[w] = True
+        sim.region[own] = ("dQ", t)
+        sim.reading[own] = True
 
-        def read_done(w=w, t=t):
-            if sim.stage[w] != ("dQ", t):
+        def read_done(t=t):
+            if sim.region[own] != ("dQ", t):
                 sim.errors.append(f"warp {w}: dQ staging of tile {t} overwritten during the reduce")
-            sim.reading[w] = False
+            sim.reading[own] = False
         sim.at(sim.lat(100, 3000), read_done)
     if sim.n_t > 0:
         yield wait(sim.drain, 0)
@@ -261,6 +312,31 @@ def test_backward_schedule_finishes_without_aliasing(n_t, stages):
         assert not sim.errors, sim.errors[:3]
 
 
+def test_each_pass_reaches_every_block_once():
+    # the compute passes and the issuer's halves name the same blocks, and each warp's
+    # dS^T stays inside the box where it alone stages dQ
+    for h in range(2):
+        assert sorted(kernel_cb(h, g) for g in range(2)) == sorted(kernel_pass_blocks(h))
+    assert sorted(kernel_cb(p, g) for p in range(2) for g in range(2)) == [0, 1, 2, 3]
+    assert all(kernel_cb(p, g) // 2 == g for p in range(2) for g in range(2))
+    kk = lambda h: [4 * (k4 // 2) + 2 * h + k4 % 2 for k4 in range(4)]   # the kernel's MMA steps
+    assert sorted({k // 2 for k in kk(0)}) == sorted(kernel_pass_blocks(0))
+    assert sorted(kk(0) + kk(1)) == list(range(8))
+
+
+def team(sim, issuer_role, compute_role):
+    nb = make_named_barrier(sim)   # one named barrier shared by the compute warps
+    return [producer(sim), issuer_role] + [compute_role(sim, w, nb) for w in range(sim.W)]
+
+
+def _finds_a_mistake(make_roles, n_t=4, stages=2, seeds=25):
+    for seed in range(seeds):
+        sim = Sim(n_t, stages, seed)
+        if not sim.run(make_roles(sim)) or sim.errors:
+            return True
+    return False
+
+
 def test_model_detects_a_planted_mistake():
     # the issuer no longer waits for s_free: the next tile's S overwrites dQ before it is read
     def bad_issuer(sim):
@@ -270,10 +346,13 @@ def test_model_detects_a_planted_mistake():
             yield wait(sim.q_full[s], t // sim.S)
 
             def mma12(t=t):
-                sim.s_cols, sim.dp_cols = ("S", t), ("dP", t)
+                sim.fill_s(("S", t))
+                for k in BLOCKS:
+                    sim.dp_cols[k] = ("dP", t)
             sim.mma(50, mma12)
             sim.commit(sim.s_full)
-            yield wait(sim.p_full, t)
+            yield wait(sim.p_full[0], t)
+            yield wait(sim.p_full[1], t)
             so = t % sim.SO
             yield wait(sim.o_full[so], t // sim.SO)
             sim.mma(50, lambda: None)
@@ -281,53 +360,90 @@ def test_model_detects_a_planted_mistake():
             sim.commit(sim.q_empty[s])
 
             def mma5(t=t):
-                sim.s_cols = ("dQ", t)
+                sim.fill_s(("dQ", t))
             sim.mma(50, mma5)
             sim.commit(sim.dq_full)
         sim.commit(sim.drain)
 
-    found = False
-    for seed in range(25):
-        sim = Sim(4, 2, seed)
-        nb = make_named_barrier(sim)
-        roles = [producer(sim), bad_issuer(sim)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
-        ok = sim.run(roles)
-        if not ok or sim.errors:
-            found = True
-            break
-    assert found
+    assert _finds_a_mistake(lambda sim: team(sim, bad_issuer(sim), compute_warp))
 
 
 def test_model_detects_a_missing_reduce_wait():
-    # a compute warp writes dS^T without waiting for its dQ reduce to read the staging
+    # a compute warp writes dS^T without waiting for its own dQ reduce to read the staging
     def bad_compute(sim, w, rows_barrier):
+        qd, g = w % 4, w // 4
+        own = (g, qd)
         for t in range(sim.n_t):
             yield from rows_barrier(t)
             yield wait(sim.s_full, t)
             yield ("delay", sim.lat(100, 800))
-            sim.stage[w] = ("dS", t)
-            sim.s_cols, sim.dp_cols, sim.ds_smem = ("P", t), ("dS", t), t
-            sim.p_full.arrive()
+            for pass_ in range(2):
+                cb = kernel_cb(pass_, g)
+                sim.s_cols[(cb, qd)], sim.dp_cols[(cb, qd)] = ("P", t), ("dS", t)
+                sim.region[(cb // 2, qd)] = ("dS", t)
+                sim.p_full[pass_].arrive()
             yield wait(sim.dq_full, t)
             yield ("delay", sim.lat(50, 500))
             sim.s_free.arrive()
-            sim.stage[w] = ("dQ", t)
-            sim.reading[w] = True
+            sim.region[own] = ("dQ", t)
+            sim.reading[own] = True
 
-            def read_done(w=w, t=t):
-                if sim.stage[w] != ("dQ", t):
+            def read_done(t=t):
+                if sim.region[own] != ("dQ", t):
                     sim.errors.append("staging overwritten")
-                sim.reading[w] = False
+                sim.reading[own] = False
             sim.at(sim.lat(1000, 5000), read_done)
         if sim.n_t > 0:
             yield wait(sim.drain, 0)
 
-    found = False
-    for seed in range(25):
-        sim = Sim(5, 2, seed)
+    assert _finds_a_mistake(lambda sim: team(sim, issuer(sim), bad_compute), n_t=5)
+
+
+def test_model_detects_a_pass_split_across_the_warps_boxes():
+    # passes that split the tile into query halves 0-63 / 64-127 instead: the warp of
+    # half 1 writes dS^T into box 0, where warp 0's dQ reduce may still be reading
+    bad_cb = lambda p, g: 2 * p + g
+    bad_blocks = lambda h: (2 * h, 2 * h + 1)
+
+    def roles(sim):
         nb = make_named_barrier(sim)
-        roles = [producer(sim), issuer(sim)] + [bad_compute(sim, w, nb) for w in range(sim.W)]
-        if not sim.run(roles) or sim.errors:
-            found = True
-            break
-    assert found
+        return [producer(sim), issuer(sim, bad_blocks)] + \
+            [compute_warp(sim, w, nb, bad_cb) for w in range(sim.W)]
+    assert _finds_a_mistake(roles, n_t=5)
+
+
+def test_model_detects_a_second_pass_issued_early():
+    # the issuer runs dV/dK of both passes after the first pass's arrivals only
+    def early_issuer(sim):
+        yield wait(sim.kv, 0)
+        for t in range(sim.n_t):
+            s = t % sim.S
+            yield wait(sim.q_full[s], t // sim.S)
+            if t > 0:
+                yield wait(sim.s_free, t - 1)
+
+            def mma1(t=t):
+                sim.fill_s(("S", t))
+                for k in BLOCKS:
+                    sim.dp_cols[k] = ("dP", t)
+            sim.mma(50, mma1)
+            so = t % sim.SO
+            yield wait(sim.o_full[so], t // sim.SO)
+            sim.commit(sim.s_full)
+            yield wait(sim.p_full[0], t)
+
+            def mma3(t=t):
+                if any(sim.s_cols[k] != ("P", t) for k in BLOCKS):
+                    sim.errors.append(f"a block of tile {t} read before it was written")
+            sim.mma(20, mma3)
+            sim.commit(sim.o_empty[so])
+            sim.commit(sim.q_empty[s])
+            yield wait(sim.p_full[1], t)
+
+            def mma5(t=t):
+                sim.fill_s(("dQ", t))
+            sim.mma(50, mma5)
+            sim.commit(sim.dq_full)
+        sim.commit(sim.drain)
+
+    assert _finds_a_mistake(lambda sim: team(sim, early_issuer(sim), compute_warp), n_t=3)
