@@ -325,24 +325,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool key_ok = k < kl;
         const float c = p.scale_log2;
         bool ok = true;
+        // query row r of tile t: its LSE and D from global memory (warps of half 0 only),
+        // fetched one tile ahead so that the loads' latency overlaps a tile's work
+        float lse_next = -INFINITY, d_next = 0.f;
+        auto fetch_rows = [&](int t) {
+            const int q = (i_lo + t) * 128 + r;
+            if (g == 0 && t < n_t && q < p.Nq) {
+                lse_next = p.lse[bh * (size_t)p.Nq + q];
+                d_next = p.dsum[bh * (size_t)p.Nq + q];
+            } else {
+                lse_next = -INFINITY;
+                d_next = 0.f;
+            }
+        };
+        fetch_rows(0);
         for (int t = 0; t < n_t; ++t) {
             const int i0 = (i_lo + t) * 128;
             float* const rb = rows + (t & 1) * 256;
-            {
-                // this thread's query row of the tile: its LSE (log2 units; +inf
-                // when the row sees no key, or lies past N_q) and D
-                const int q = i0 + r;
-                float l2 = INFINITY, dd = 0.f;
-                if (q < p.Nq) {
-                    const float L = p.lse[bh * (size_t)p.Nq + q];
-                    l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
-                    dd = p.dsum[bh * (size_t)p.Nq + q];
-                }
-                if (g == 0) {
-                    rb[r] = l2;
-                    rb[128 + r] = dd;
-                }
+            if (g == 0) {
+                // the row's LSE in log2 units (+inf when the row sees no key, or lies
+                // past N_q) and D
+                rb[r] = (lse_next == -INFINITY) ? INFINITY : lse_next * 1.4426950408889634f;
+                rb[128 + r] = d_next;
             }
+            fetch_rows(t + 1);
             // all four warps wrote the tile's row data; leave together if any gave up
             if (named_bar_or(kBwdBarCompute, 32 * kBwdComputeWarps, !ok)) break;
             bool good = wait_bounded(bar_s_full, (uint32_t)(t & 1), abort_flag, p.wait_limit);

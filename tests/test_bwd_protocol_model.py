@@ -11,6 +11,8 @@ latencies are drawn for copies, MMAs and compute.  Checked for every schedule:
   * the data each role consumes is the data of its own tile (Q/dO slot contents,
     S/dP contents, the dS^T buffer and the dQ columns), so no buffer is overwritten
     while still in use.
+An alternative issue order -- dP^T of tile t + 1 right after dQ_t, ahead of the wait for
+the compute warps to read dQ_t out of the S columns -- is checked as well.
 Geometry as in the kernel: warp w serves TMEM lane quadrant qd and query half g; the
 tile's 128 queries are four blocks cb of 32.  A warp computes its blocks cb = 2g + pass
 in two passes and hands each pass over on p_full[pass]; the issuer runs dV and dK of
@@ -188,10 +190,31 @@ def producer(sim):
         yield ("delay", 1)
 
 
-def issuer(sim, pass_blocks=kernel_pass_blocks):
+def issuer(sim, pass_blocks=kernel_pass_blocks, dp_ahead=False, dp_too_early=False):
+    """The kernel's order: S^T_t, then dP^T_t once dO_t has landed.  dp_ahead: dP^T of
+    tile t + 1 right after dQ_t instead, before the wait for s_free (also safe; measured
+    slower).  dp_too_early (a planted mistake): dP^T of tile t + 1 right after tile t's
+    s_full commit."""
+    def issue_dp(t):
+        so = t % sim.SO
+        yield wait(sim.o_full[so], t // sim.SO)
+
+        def mma2(t=t, so=so):
+            if sim.oslot[so] != t:
+                sim.errors.append(f"dP of tile {t} read dO slot holding {sim.oslot[so]}")
+            for k in BLOCKS:
+                if sim.dp_cols[k] not in (None, ("dS", t - 1)):
+                    sim.errors.append(f"dP of tile {t} overwrote {sim.dp_cols[k]}")
+                sim.dp_cols[k] = ("dP", t)
+        sim.mma(sim.lat(50, 150), mma2)
+
     yield wait(sim.kv, 0)
+    dp_ahead = dp_ahead and not dp_too_early
+    if dp_ahead and sim.n_t > 0:
+        yield from issue_dp(0)
     for t in range(sim.n_t):
         s = t % sim.S
+        so = t % sim.SO
         yield wait(sim.q_full[s], t // sim.S)
         if t > 0:
             yield wait(sim.s_free, t - 1)
@@ -201,16 +224,11 @@ def issuer(sim, pass_blocks=kernel_pass_blocks):
                 sim.errors.append(f"S of tile {t} read Q slot holding {sim.slot[s]}")
             sim.fill_s(("S", t))
         sim.mma(sim.lat(50, 150), mma1)
-        so = t % sim.SO
-        yield wait(sim.o_full[so], t // sim.SO)
-
-        def mma2(t=t, so=so):
-            if sim.oslot[so] != t:
-                sim.errors.append(f"dP of tile {t} read dO slot holding {sim.oslot[so]}")
-            for k in BLOCKS:
-                sim.dp_cols[k] = ("dP", t)
-        sim.mma(sim.lat(50, 150), mma2)
+        if not dp_ahead:
+            yield from issue_dp(t)
         sim.commit(sim.s_full)
+        if dp_too_early and t + 1 < sim.n_t:
+            yield from issue_dp(t + 1)
         for h in range(2):
             yield wait(sim.p_full[h], t)
             keys = [(cb, qd) for cb in pass_blocks(h) for qd in range(4)]
@@ -234,6 +252,8 @@ def issuer(sim, pass_blocks=kernel_pass_blocks):
             sim.fill_s(("dQ", t))
         sim.mma(sim.lat(50, 200), mma5)
         sim.commit(sim.dq_full)
+        if dp_ahead and t + 1 < sim.n_t:
+            yield from issue_dp(t + 1)
         yield ("delay", 1)
     sim.commit(sim.drain)
 
@@ -303,11 +323,12 @@ def make_named_barrier(sim):
 
 @pytest.mark.parametrize("n_t", [1, 2, 3, 7])
 @pytest.mark.parametrize("stages", [(1, 1), (2, 2), (2, 1)])
-def test_backward_schedule_finishes_without_aliasing(n_t, stages):
+@pytest.mark.parametrize("dp_ahead", [True, False])
+def test_backward_schedule_finishes_without_aliasing(n_t, stages, dp_ahead):
     for seed in range(25):
         sim = Sim(n_t, stages[0], seed, stages_o=stages[1])
         nb = make_named_barrier(sim)
-        roles = [producer(sim), issuer(sim)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
+        roles = [producer(sim), issuer(sim, dp_ahead=dp_ahead)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
         assert sim.run(roles), f"deadlock (n_t={n_t}, stages={stages}, seed={seed})"
         assert not sim.errors, sim.errors[:3]
 
@@ -447,3 +468,11 @@ def test_model_detects_a_second_pass_issued_early():
         sim.commit(sim.drain)
 
     assert _finds_a_mistake(lambda sim: team(sim, early_issuer(sim), compute_warp), n_t=3)
+
+
+def test_model_detects_the_next_dp_issued_before_dp_is_read():
+    def roles(sim):
+        nb = make_named_barrier(sim)
+        return [producer(sim), issuer(sim, dp_too_early=True)] + \
+            [compute_warp(sim, w, nb) for w in range(sim.W)]
+    assert _finds_a_mistake(roles, n_t=4, stages=2)
