@@ -81,17 +81,22 @@ struct BwdCfg {
     static constexpr int kRowOff = kDQ2Off + (D == 128 ? 2 * kSwizzleBoxBytes : 0);   // [2][lse2 x128 | D x128] fp32
     static constexpr int kBarOff = kRowOff + 2 * 256 * 4;
     // barriers: kv_full, q_full[SQ], q_empty[SQ], o_full[SO], o_empty[SO], s_full,
-    // p_full (pass 0), dq_full, s_free, drain, p_full (pass 1)
-    static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesO + 6;
+    // p_full (pass 0), dq_full, s_free, drain, p_full (pass 1), kv_tmem
+    static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesO + 7;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
     static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA on sm_100");
     // TMEM columns: S^T (then P^T as bf16, then dQ) at 0; dP^T (then dS^T) at 128;
-    // dV at 256; dK at 256 + D.  P^T of queries 0-63 sits at columns 0-31 and of
-    // queries 64-127 at 64-95 (dS^T likewise from 128), so each compute warp
-    // overwrites only columns it has itself read.
+    // dV at 256; dK at 256 + D.  P^T of the 32 queries 32cb.. sits at columns
+    // 32cb..32cb+15 (dS^T likewise from 128), so each compute warp overwrites only
+    // columns it has itself read.  At d = 64 the block's K and V rows (bf16 pairs)
+    // also live in TMEM, at 384 and 416: S^T and dP^T then take their A operand from
+    // TMEM and read only Q / dO from shared memory.
+    static constexpr bool kKVInTmem = (D == 64);
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
-    static_assert(kColDK + D <= 512, "TMEM columns");
+    static constexpr uint32_t kColK = 384, kColV = 384 + D / 2;
+    static_assert(kColDK + D <= (kKVInTmem ? kColK : 512u) && (!kKVInTmem || kColV + D / 2 <= 512u),
+                  "TMEM columns");
     // Instruction descriptors (kind::f16, D = f32, A = B = bf16, M = 128):
     //   S^T, dP^T: A K-major, B K-major, N = 128 (queries);
     //   dV, dK:    A from TMEM, B MN-major (dO / Q rows are queries), N = D;
@@ -142,6 +147,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t bar_dq_full = bar(kB0 + 2);
     const uint32_t bar_s_free = bar(kB0 + 3);
     const uint32_t bar_drain = bar(kB0 + 4);
+    const uint32_t bar_kv_tmem = bar(kB0 + 6);   // K and V rows copied into TMEM (d = 64)
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
     float* const rows = reinterpret_cast<float*>(base_ptr + C::kRowOff);
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_dq_full, 1);
         mbar_init(bar_s_free, kBwdComputeWarps);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_kv_tmem, kBwdComputeWarps);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_q);
@@ -246,6 +253,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ============================================================ MMA issuer
         if (lane == 0 && n_t > 0) {
             bool ok = wait_bounded(bar_kv, 0, abort_flag, p.wait_limit);
+            if (C::kKVInTmem && ok) ok = wait_bounded(bar_kv_tmem, 0, abort_flag, p.wait_limit);
             const uint32_t k_s = base + C::kKOff, v_s = base + C::kVOff, ds_s = base + C::kDSOff;
             for (int t = 0; t < n_t && ok; ++t) {
                 const int sq = t % C::kStagesQ, so = t % C::kStagesO;
@@ -259,8 +267,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
                     const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
-                    umma_ss(tmem + C::kColS, smem_desc_sw128(k_s + koff, 16, 1024), smem_desc_sw128(q_s + koff, 16, 1024),
-                            C::kIdescST, kk > 0 ? 1u : 0u);
+                    if constexpr (C::kKVInTmem)
+                        umma_ts(tmem + C::kColS, tmem + C::kColK + 8u * (uint32_t)kk,
+                                smem_desc_sw128(q_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
+                    else
+                        umma_ss(tmem + C::kColS, smem_desc_sw128(k_s + koff, 16, 1024),
+                                smem_desc_sw128(q_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
                 }
                 // dO_i may land after Q_i (its slot frees when the previous tile's dV is done)
                 ok = wait_bounded(bar_o_full(so), (uint32_t)((t / C::kStagesO) & 1), abort_flag, p.wait_limit);
@@ -269,8 +281,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
                     const uint32_t koff = (uint32_t)((kk / 4) * kSwizzleBoxBytes + (kk % 4) * 32);
-                    umma_ss(tmem + C::kColDP, smem_desc_sw128(v_s + koff, 16, 1024),
-                            smem_desc_sw128(do_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
+                    if constexpr (C::kKVInTmem)
+                        umma_ts(tmem + C::kColDP, tmem + C::kColV + 8u * (uint32_t)kk,
+                                smem_desc_sw128(do_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
+                    else
+                        umma_ss(tmem + C::kColDP, smem_desc_sw128(v_s + koff, 16, 1024),
+                                smem_desc_sw128(do_s + koff, 16, 1024), C::kIdescST, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar_s_full);
                 // dV and dK for the queries of each pass as soon as the compute warps
@@ -339,6 +355,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         };
         fetch_rows(0);
+        if (C::kKVInTmem && n_t > 0) {
+            // key row r of K (warps of half 0) or V (half 1) from the swizzled tile
+            // (16-byte chunk c of row r at c ^ (r % 8)) into this lane's TMEM row: column
+            // j holds elements 2j and 2j + 1, the A-operand layout of the MMAs
+            const bool good = wait_bounded(bar_kv, 0, abort_flag, p.wait_limit);
+            if (__all_sync(0xffffffffu, good)) {
+                const uint32_t src = base + (g == 0 ? C::kKOff : C::kVOff) + (uint32_t)(r * 128);
+                uint32_t w[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[4 * c4]), "=r"(w[4 * c4 + 1]), "=r"(w[4 * c4 + 2]), "=r"(w[4 * c4 + 3])
+                                 : "r"(src + (uint32_t)((c4 ^ (r & 7)) << 4))
+                                 : "memory");
+                tmem_st32(tmem + lane_off + (g == 0 ? C::kColK : C::kColV), w);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_kv_tmem);
+            } else {
+                ok = false;
+            }
+        }
         for (int t = 0; t < n_t; ++t) {
             const int i0 = (i_lo + t) * 128;
             float* const rb = rows + (t & 1) * 256;

@@ -11,6 +11,8 @@ latencies are drawn for copies, MMAs and compute.  Checked for every schedule:
   * the data each role consumes is the data of its own tile (Q/dO slot contents,
     S/dP contents, the dS^T buffer and the dQ columns), so no buffer is overwritten
     while still in use.
+At d = 64 the compute warps first copy the block's K and V rows into TMEM and arrive on
+kv_tmem, which the issuer waits for before the first S^T.
 An alternative issue order -- dP^T of tile t + 1 right after dQ_t, ahead of the wait for
 the compute warps to read dQ_t out of the S columns -- is checked as well.
 Geometry as in the kernel: warp w serves TMEM lane quadrant qd and query half g; the
@@ -66,8 +68,9 @@ REGIONS = [(box, qd) for box in range(2) for qd in range(4)]
 
 
 class Sim:
-    def __init__(self, n_t, stages, seed, warps=8, stages_o=None):
+    def __init__(self, n_t, stages, seed, warps=8, stages_o=None, kv_in_tmem=False):
         self.rng = random.Random(seed)
+        self.kv_in_tmem = kv_in_tmem
         self.n_t, self.S, self.W = n_t, stages, warps
         self.SO = stages if stages_o is None else stages_o
         self.now = 0
@@ -83,6 +86,9 @@ class Sim:
         self.p_full = [b(f"p_full{h}", warps) for h in range(2)]
         self.dq_full, self.s_free = b("dq_full", 1), b("s_free", warps)
         self.drain = b("drain", 1)
+        self.kv_tmem = b("kv_tmem", warps)   # K and V rows copied into TMEM (d = 64)
+        self.k_tmem = None                   # what the TMEM copy of K / V was taken from
+        self.kv_landed = False
         # buffer contents: which tile's data they hold
         self.slot = [None] * stages           # Q slot -> tile
         self.oslot = [None] * self.SO         # dO slot -> tile
@@ -171,7 +177,10 @@ def wait(bar, k):
 
 
 def producer(sim):
-    sim.at(sim.lat(50, 400), sim.kv.arrive)
+    def land_kv():
+        sim.kv_landed = True
+        sim.kv.arrive()
+    sim.at(sim.lat(50, 400), land_kv)
     for t in range(sim.n_t):
         s = t % sim.S
         yield wait(sim.q_empty[s], t // sim.S - 1)
@@ -209,6 +218,10 @@ def issuer(sim, pass_blocks=kernel_pass_blocks, dp_ahead=False, dp_too_early=Fal
         sim.mma(sim.lat(50, 150), mma2)
 
     yield wait(sim.kv, 0)
+    if sim.kv_in_tmem:
+        yield wait(sim.kv_tmem, 0)
+        if sim.k_tmem != "copied":
+            sim.errors.append("S^T issued before K and V were copied into TMEM")
     dp_ahead = dp_ahead and not dp_too_early
     if dp_ahead and sim.n_t > 0:
         yield from issue_dp(0)
@@ -261,6 +274,15 @@ def issuer(sim, pass_blocks=kernel_pass_blocks, dp_ahead=False, dp_too_early=Fal
 def compute_warp(sim, w, rows_barrier, cb_of=kernel_cb):
     qd, g = w % 4, w // 4
     own = (g, qd)                       # where this warp stages dQ
+    if sim.kv_in_tmem and sim.n_t > 0:
+        yield wait(sim.kv, 0)
+        if not sim.kv_landed:
+            sim.errors.append(f"warp {w} copied K/V into TMEM before they landed")
+        yield ("delay", sim.lat(20, 200))
+        sim.copies = getattr(sim, "copies", 0) + 1
+        if sim.copies == sim.W:
+            sim.k_tmem = "copied"
+        sim.kv_tmem.arrive()
     for t in range(sim.n_t):
         yield from rows_barrier(t)
         yield wait(sim.s_full, t)
@@ -326,7 +348,8 @@ def make_named_barrier(sim):
 @pytest.mark.parametrize("dp_ahead", [True, False])
 def test_backward_schedule_finishes_without_aliasing(n_t, stages, dp_ahead):
     for seed in range(25):
-        sim = Sim(n_t, stages[0], seed, stages_o=stages[1])
+        # d = 64 (two Q and dO slots) keeps K and V in TMEM as well
+        sim = Sim(n_t, stages[0], seed, stages_o=stages[1], kv_in_tmem=stages == (2, 2))
         nb = make_named_barrier(sim)
         roles = [producer(sim), issuer(sim, dp_ahead=dp_ahead)] + [compute_warp(sim, w, nb) for w in range(sim.W)]
         assert sim.run(roles), f"deadlock (n_t={n_t}, stages={stages}, seed={seed})"
