@@ -164,12 +164,12 @@ struct Cfg {
     static constexpr int kPBufs = 3;                             // TMEM probability buffers
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S],
     // s_full[2 (per softmax warp)], s_free[2], p_full[3], pv_done[3],
-    // m_ready[4 quadrants][2], drain
+    // 8 unused slots (the reference max now travels in tagged words), drain
     static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 3 + 3 + 8 + 1;
     static_assert(kSBufs <= 2 && kPBufs <= 3, "barrier slots");
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;      // tmem base, abort flag
-    static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row]
-    static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 4;  // epilogue exchange: m, lu [2][row] each
+    static constexpr int kMrefOff = kMiscOff + 16;               // published reference max [group][row], 8 B each
+    static constexpr int kEpiOff = kMrefOff + kGroups * kBlockM * 8;  // epilogue exchange: m, lu [2][row] each
     static constexpr int kSmemUsed = kEpiOff + 2 * kGroups * kBlockM * 4 + 1024;  // + alignment slack
     // One CTA per SM either way (it holds all 512 TMEM columns), so the smaller
     // E4M3 layouts reserve as much shared memory as the bf16 d = 64 one.
@@ -235,6 +235,39 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
             return false;
         }
     }
+}
+
+// The reference max one softmax warp hands to the other warp of its lane quadrant,
+// per row: one 64-bit shared word {tile index (high half), max bits (low half)},
+// written and read in single accesses, so a reader that sees the tile it waits for
+// also sees that tile's max.  The reader polls until the word names its tile (the
+// writer cannot move on to a later tile before it has read this reader's next word).
+__device__ __forceinline__ unsigned long long ld_relaxed_shared_u64(uint32_t addr) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.cta.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_shared_u64(uint32_t addr, unsigned long long v) {
+    asm volatile("st.relaxed.cta.shared.b64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_tagged_max(uint32_t addr, uint32_t tag, float& m, volatile int* abort_flag,
+                                                unsigned long long limit) {
+    unsigned long long v = ld_relaxed_shared_u64(addr);
+    if ((uint32_t)(v >> 32) != tag) {
+        const long long t0 = clock64();
+        while (true) {
+            v = ld_relaxed_shared_u64(addr);
+            if ((uint32_t)(v >> 32) == tag) break;
+            if (*abort_flag) return false;
+            if ((unsigned long long)(clock64() - t0) > limit) {
+                *abort_flag = 1;
+                atomicExch(&g_fa_status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+    m = __uint_as_float((uint32_t)v);
+    return true;
 }
 
 // Bounded wait for this thread's own asynchronous work (a TMA copy it issued, or
@@ -450,11 +483,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     auto bar_s_free = [&](int b) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + b); };
     auto bar_p_full = [&](int b) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + b); };
     auto bar_pv_done = [&](int b) { return base + C::kBarOff + 8u * (8 + 2 * C::kStages + b); };
-    auto bar_m_ready = [&](int qd, int g) { return base + C::kBarOff + 8u * (11 + 2 * C::kStages + 2 * qd + g); };
     const uint32_t bar_drain = base + C::kBarOff + 8u * (19 + 2 * C::kStages);
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
-    float* const mref = reinterpret_cast<float*>(base_ptr + C::kMrefOff);     // [group][row]
+    // [group][row]: {tile, reference max} words (wait_tagged_max)
+    const uint32_t mref_w = base + C::kMrefOff;
     float* const epi = reinterpret_cast<float*>(base_ptr + C::kEpiOff);       // m, l, lu [group][row] each
     const uint32_t q_tile = base + C::kQOff;
     auto ring_slot = [&](int r, int s) {
@@ -550,7 +583,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             mbar_init(bar_p_full(b2), 4);   // one arrival per lane quadrant
             mbar_init(bar_pv_done(b2), 1);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(bar_m_ready(i >> 1, i & 1), 1);
         mbar_init(bar_drain, 2);   // one commit from each MMA issuer
         *abort_flag = 0;
         fence_mbar_init();
@@ -559,6 +591,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_o);
     }
+    // no reference max published yet: tag 0xffffffff names no tile
+    for (int i = threadIdx.x; i < kGroups * kBlockM; i += kNumThreads)
+        st_relaxed_shared_u64(mref_w + 8u * (uint32_t)i, ~0ull);
     if (warp == kMmaWarp) {
         tmem_alloc(smem_addr(tmem_holder), kTmemCols);
         tmem_relinquish();
@@ -769,21 +804,18 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // reference max after tile j-1, published by the other warp of the quadrant
             float m_prev = -INFINITY;
             if (j > 0) {
-                good = wait_bounded(bar_m_ready(qd, g ^ 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag,
-                                    p.wait_limit);
+                good = wait_tagged_max(mref_w + 8u * (uint32_t)((g ^ 1) * kBlockM + r), (uint32_t)(j - 1), m_prev,
+                                       abort_flag, p.wait_limit);
                 if (!__all_sync(0xffffffffu, good)) {
                     ok = false;
                     break;
                 }
-                m_prev = mref[(g ^ 1) * kBlockM + r];
             }
             const float t_max = mx * cs;  // cs > 0, so -inf stays -inf
             const float m_cur = (t_max > m_prev + kRescaleThreshold) ? t_max : m_prev;
-            if (j + 1 < n_kv) {
-                mref[g * kBlockM + r] = m_cur;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_m_ready(qd, g));
-            }
+            if (j + 1 < n_kv)
+                st_relaxed_shared_u64(mref_w + 8u * (uint32_t)(g * kBlockM + r),
+                                      ((unsigned long long)(uint32_t)j << 32) | __float_as_uint(m_cur));
             if (m_cur != m_seen) {
                 const float f = ex2_approx(m_seen - m_cur);  // 0 while m_seen is -inf
                 lu *= f;

@@ -125,7 +125,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     auto bar_s_free = [&](int b) { return base + C::kBarOff + 8u * (3 + 2 * C::kStages + b); };
     auto bar_p_full = [&](int b) { return base + C::kBarOff + 8u * (5 + 2 * C::kStages + b); };
     auto bar_pv_done = [&](int b) { return base + C::kBarOff + 8u * (8 + 2 * C::kStages + b); };
-    auto bar_m_ready = [&](int qd, int g) { return base + C::kBarOff + 8u * (11 + 2 * C::kStages + 2 * qd + g); };
     // the persistent kernel's own
     const uint32_t bar_q_free = base + PC::kExtraOff;            // QK^T products of a block have read Q
     const uint32_t bar_o_free = base + PC::kExtraOff + 8;        // O and its row sums read out of TMEM
@@ -139,7 +138,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     int* const mailbox = reinterpret_cast<int*>(base_ptr + PC::kMailOff);
     uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
-    float* const mref = reinterpret_cast<float*>(base_ptr + C::kMrefOff);     // [parity][row]
+    // [parity][row]: {tile over all blocks, reference max} words (wait_tagged_max)
+    const uint32_t mref_w = base + C::kMrefOff;
     float* const epi2 = reinterpret_cast<float*>(base_ptr + PC::kEpiOff);     // [block parity][m, lu][parity][row]
     const uint32_t q_tile = base + C::kQOff;
     auto ring_slot = [&](int r, int s) {
@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             mbar_init(bar_p_full(b2), 4);
             mbar_init(bar_pv_done(b2), 1);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(bar_m_ready(i >> 1, i & 1), 1);
         mbar_init(bar_q_free, 1);
         mbar_init(bar_o_free, kSoftmaxWarps);
         mbar_init(bar_drain, 1);
@@ -196,6 +195,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t a = ring_slot(1, sl) + (uint32_t)C::kTileBytes + (uint32_t)(i % (C::kBoxBytes / 16)) * 16u;
         asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(C::kOnesWord) : "memory");
     }
+    // no reference max published yet: tag 0xffffffff names no tile
+    for (int i = threadIdx.x; i < kGroups * kBlockM; i += kNumThreads)
+        st_relaxed_shared_u64(mref_w + 8u * (uint32_t)i, ~0ull);
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
@@ -415,7 +417,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         int tt0 = 0;                 // tiles of the blocks before this one
         int nq = 0;                  // blocks with K/V tiles so far
         int sf_own = 0;              // completions of s_full(g) before this block
-        int mr_other = 0;            // publications on m_ready(qd, g ^ 1) before this block
         for (int k = 0;; ++k) {
             const int n_kv = it.n_kv;
             const int h = it.h, b = it.b, m0 = it.m0, off = it.off, t0 = it.t0;
@@ -483,23 +484,21 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
                 const float mx = fmaxf(fmaxf(chunk_max32(s, 0), chunk_max32(s, 32)),
                                        fmaxf(chunk_max32(s, 64), chunk_max32(s, 96)));
+                // the other warp's reference max after tile tt - 1 (same block)
                 float m_prev = -INFINITY;
                 if (j > 0) {
-                    good = wait_bounded(bar_m_ready(qd, g ^ 1), (uint32_t)((mr_other + ((j - 1) >> 1)) & 1),
-                                        abort_flag, p.wait_limit);
+                    good = wait_tagged_max(mref_w + 8u * (uint32_t)((g ^ 1) * kBlockM + r), (uint32_t)(tt - 1),
+                                           m_prev, abort_flag, p.wait_limit);
                     if (!__all_sync(0xffffffffu, good)) {
                         ok = false;
                         break;
                     }
-                    m_prev = mref[(g ^ 1) * kBlockM + r];
                 }
                 const float t_max = mx * cs;
                 const float m_cur = (t_max > m_prev + kRescaleThreshold) ? t_max : m_prev;
-                if (j + 1 < n_kv) {
-                    mref[g * kBlockM + r] = m_cur;
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_m_ready(qd, g));
-                }
+                if (j + 1 < n_kv)
+                    st_relaxed_shared_u64(mref_w + 8u * (uint32_t)(g * kBlockM + r),
+                                          ((unsigned long long)(uint32_t)tt << 32) | __float_as_uint(m_cur));
                 if (m_cur != m_seen) {
                     const float f = ex2_approx(m_seen - m_cur);
                     lu *= f;
@@ -627,10 +626,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // the counters of the blocks taken so far
             if (n_kv > 0) {
                 tt0 += n_kv;
-                // group 0 takes the even tiles and publishes a reference max on
-                // every one but the last tile; group 1 the odd ones
+                // group 0 takes the even tiles, group 1 the odd ones
                 sf_own += (g == 0) ? (n_kv + 1) / 2 : n_kv / 2;
-                mr_other += (g == 0) ? (n_kv - 1) / 2 : n_kv / 2;
                 ++nq;
             }
             if (nxt <= 0) break;   // the same answer in both warps (same mailbox slot)

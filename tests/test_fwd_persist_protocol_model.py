@@ -19,14 +19,16 @@ Checked for every schedule:
     PV(t); the first PV of a block (which starts O afresh) runs only after all eight
     softmax warps read the previous block's O; the epilogue reads O after every PV of
     its block; the epilogue exchange buffer is not overwritten before the partner
-    warp read it; every mailbox reader gets the item of its own block.
+    warp read it; every mailbox reader gets the item of its own block; the reference
+    max travels between the two warps of a quadrant in a word tagged with the tile's
+    index over all blocks, which is read before it is overwritten.
 """
 import random
 
 import pytest
 
 from test_bwd_protocol_model import Barrier
-from test_fwd_protocol_model import Fwd, wait
+from test_fwd_protocol_model import Fwd, publish_max, take_max, wait
 
 
 class Persist(Fwd):
@@ -213,7 +215,7 @@ def pv_issuer(m):
 
 
 def softmax(m, q, g):
-    k, tt0, nq, sf_own, mr_other, n_epi = 0, 0, 0, 0, 0, 0
+    k, tt0, nq, sf_own, n_epi = 0, 0, 0, 0, 0
     while True:
         n = m.n_of(k)
         for j in range(g, n, 2):
@@ -225,13 +227,11 @@ def softmax(m, q, g):
             yield ("delay", m.lat(100, 300) * m.slow)
             m.s_reads[sb] += 1
             m.s_free[sb].arrive()
+            yield ("delay", m.lat(20, 600) * m.slow)   # mask and row max of the scores
             if j > 0:
-                yield wait(m.m_ready[q][g ^ 1], mr_other + ((j - 1) >> 1))
-                if m.mref.get((q, g ^ 1)) != (k, j - 1):
-                    m.errors.append(f"q{q} block {k} tile {j} read the max of {m.mref.get((q, g ^ 1))}")
+                yield from take_max(m, q, g, tt)   # the other warp's tile tt - 1 (same block)
             if j + 1 < n:
-                m.mref[(q, g)] = (k, j)
-                m.m_ready[q][g].arrive()
+                publish_max(m, q, g, tt)
             pb = tt % m.n_p
             if tt >= m.n_p:
                 yield wait(m.pv_done[pb], (tt - m.n_p) // m.n_p)
@@ -274,7 +274,6 @@ def softmax(m, q, g):
             m.o_free.arrive()
             tt0 += n
             sf_own += (n + 1) // 2 if g == 0 else n // 2
-            mr_other += (n - 1) // 2 if g == 0 else n // 2
             nq += 1
         if nxt is None:
             return

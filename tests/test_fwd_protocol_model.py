@@ -15,6 +15,11 @@ Checked for every schedule:
     only after PV(j-3) finished reading that P buffer and PV(j) reads P(j) complete;
     an O rescale at tile j runs after PV(j-1) and before PV(j); the epilogue reads O
     after every PV.
+The reference max of tile j goes from warp (q, g) to warp (q, g ^ 1) in a shared word
+tagged with j, written in one store; the reader polls until the tag names the tile it
+needs.  Checked as well: the reader gets that tile's max, and no word is overwritten
+before its reader took it (a warp reads the other's word for tile j - 1 before it
+publishes tile j).  A planted writer that publishes before it reads is caught.
 """
 import random
 
@@ -40,7 +45,6 @@ class Fwd:
         self.s_free = [b(f"s_free{i}", 4) for i in range(n_s)]
         self.p_full = [b(f"p_full{i}", 4) for i in range(n_p)]
         self.pv_done = [b(f"pv_done{i}", 1) for i in range(n_p)]
-        self.m_ready = [[b(f"m_ready{q}{g}", 1) for g in range(2)] for q in range(4)]
         self.drain = b("drain", 2)
         self.kslot, self.vslot = [None] * ns_k, [None] * ns_v
         self.s_buf = [None] * n_s        # tile held by each score buffer
@@ -48,7 +52,8 @@ class Fwd:
         self.p_buf = [None] * n_p        # (tile, quadrants written)
         self.pv_done_count = 0           # PVs finished
         self.pv_started = -1             # last PV started
-        self.mref = {}                   # (q, g) -> tile whose max it holds
+        self.word = {}                   # (q, g) -> tile tag of the published max
+        self.word_read = {}              # (q, g) -> last tag the other warp took
         self.errors = []
 
     def at(self, dt, fn):
@@ -191,7 +196,33 @@ def pv_issuer(m):
     m.commit(m.drain)
 
 
-def softmax(m, q, g):
+def take_max(m, q, g, j):
+    # poll the other warp's word until it carries tile j - 1
+    polls = 0
+    while m.word.get((q, g ^ 1)) != j - 1:
+        polls += 1
+        assert polls < 10 ** 5, "poll never satisfied"
+        yield ("delay", m.lat(5, 40))
+    m.word_read[(q, g ^ 1)] = j - 1
+
+
+def publish_max(m, q, g, j):
+    prev = m.word.get((q, g))
+    if prev is not None and m.word_read.get((q, g)) != prev:
+        m.errors.append(f"q{q}: max of tile {prev} overwritten by tile {j} before it was read")
+    m.word[(q, g)] = j
+
+
+def exchange_max(m, q, g, j, publish_first=False):
+    if publish_first and j + 1 < m.n:
+        publish_max(m, q, g, j)
+    if j > 0:
+        yield from take_max(m, q, g, j)
+    if not publish_first and j + 1 < m.n:
+        publish_max(m, q, g, j)
+
+
+def softmax(m, q, g, publish_first=False):
     for j in range(g, m.n, 2):
         yield wait(m.s_full[g], j >> 1)
         sb = j % m.n_s
@@ -200,13 +231,8 @@ def softmax(m, q, g):
         yield ("delay", m.lat(100, 300) * m.slow)
         m.s_reads[sb] += 1
         m.s_free[sb].arrive()
-        if j > 0:
-            yield wait(m.m_ready[q][g ^ 1], (j - 1) >> 1)
-            if m.mref.get((q, g ^ 1)) != j - 1:
-                m.errors.append(f"q{q} tile {j} read the max of tile {m.mref.get((q, g ^ 1))}")
-        if j + 1 < m.n:
-            m.mref[(q, g)] = j
-            m.m_ready[q][g].arrive()
+        yield ("delay", m.lat(20, 600) * m.slow)   # mask and row max of the scores
+        yield from exchange_max(m, q, g, j, publish_first)
         pb = j % m.n_p
         if j >= m.n_p:
             yield wait(m.pv_done[pb], (j - m.n_p) // m.n_p)
@@ -252,11 +278,7 @@ def test_model_detects_a_planted_mistake():
             yield ("delay", m.lat(100, 300))
             m.s_reads[0] += 1
             m.s_free[0].arrive()
-            if j > 0:
-                yield wait(m.m_ready[q][g ^ 1], (j - 1) >> 1)
-            if j + 1 < m.n:
-                m.mref[(q, g)] = j
-                m.m_ready[q][g].arrive()
+            yield from exchange_max(m, q, g, j)
             pb = j % 3
             yield ("delay", m.lat(50, 200))
             cur = m.p_buf[pb]
@@ -271,6 +293,24 @@ def test_model_detects_a_planted_mistake():
         roles = [k_producer(m), v_producer(m), qk_issuer(m), pv_issuer(m)]
         roles += [bad_softmax(m, q, g) for q in range(4) for g in range(2)]
         if not m.run(roles) or m.errors:
+            caught = True
+            break
+    assert caught
+
+
+def test_model_detects_a_max_published_before_the_other_is_read():
+    # a warp that publishes tile j's max before taking the other warp's tile j - 1:
+    # the other warp can then publish j + 1 over the word this one has not read yet
+    caught = False
+    for seed in range(40):
+        m = Fwd(9, 2, 2, seed, slow=3.0)
+        roles = [k_producer(m), v_producer(m), qk_issuer(m), pv_issuer(m)]
+        roles += [softmax(m, q, g, publish_first=True) for q in range(4) for g in range(2)]
+        try:
+            ok = m.run(roles)
+        except AssertionError:
+            ok = False
+        if not ok or m.errors:
             caught = True
             break
     assert caught
