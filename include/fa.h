@@ -417,6 +417,25 @@ FA_API int fa_selftest_fwd_timeout(const void *q, const void *k, const void *v, 
                                    fa_stream_t stream);
 
 /*
+ * fa_selftest_bwd_timeout -- failure-detection self test of the backward
+ * kernel's wind-down.  Runs fa_bwd (arguments as fa_bwd, no key_lens) with
+ * every pipeline wait of the main kernel bounded by `limit_cycles` SM clock
+ * cycles (1 .. 2^32) instead of about a second, synchronises `stream` and
+ * returns what fa_get_device_status reports.  With a limit of a few cycles
+ * some wait runs out: every role of that CTA stops after waiting (with the
+ * default limit, ignoring the abort) for the copies, MMAs and tensor
+ * reduce-adds it has already issued, so nothing lands in released shared
+ * memory or TMEM; the call returns FA_ERR_DEVICE_TIMEOUT and the CUDA context
+ * stays usable.  dq, dk and dv then hold unspecified values.  B, H, N_q and N_k
+ * must be > 0 (otherwise nothing would wait: FA_ERR_INVALID_ARG).
+ */
+FA_API int fa_selftest_bwd_timeout(const void *q, const void *k, const void *v, const void *o,
+                                   const float *lse, const void *dout, void *dq, void *dk,
+                                   void *dv, int B, int H, int N_q, int N_k, int d, float scale,
+                                   int causal, void *workspace, size_t workspace_bytes,
+                                   unsigned long long limit_cycles, fa_stream_t stream);
+
+/*
  * fa_last_error -- the CUDA call and error text behind the most recent
  * FA_ERR_CUDA returned on the calling thread ("" if none).  The string
  * belongs to the library and stays valid until the thread's next failing call.

@@ -12,7 +12,7 @@ from .binding import (  # noqa: F401
     fa_fwd_host, fa_fwd_host_workspace_size, fa_bwd, fa_bwd_workspace_size, fa_fwd_splitkv, fa_fwd_splitkv_noalloc,
     fa_fwd_splitkv_workspace_size, fa_fwd_window, fa_fwd_bias, fa_fwd_bias_table, fa_fwd_fp8, fa_fwd_varlen,
     fa_splitkv_num_splits, fa_get_device_status, fa_selftest_wait_timeout,
-    fa_selftest_fwd_timeout,
+    fa_selftest_fwd_timeout, fa_selftest_bwd_timeout,
     fa_status_string, fa_last_error,
     fa_version, library_path, load_library,
 )

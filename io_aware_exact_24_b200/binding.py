@@ -99,6 +99,9 @@ def load_library() -> ctypes.CDLL:
             lib.fa_selftest_fwd_timeout.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                     f32, i32, ctypes.c_ulonglong, vp]
             lib.fa_selftest_fwd_timeout.restype = i32
+            lib.fa_selftest_bwd_timeout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                                    i32, i32, f32, i32, vp, sz, ctypes.c_ulonglong, vp]
+            lib.fa_selftest_bwd_timeout.restype = i32
             lib.fa_last_error.argtypes = []
             lib.fa_last_error.restype = ctypes.c_char_p
             lib.fa_version.argtypes = []
@@ -294,6 +297,15 @@ def fa_selftest_fwd_timeout(q, k, v, o, lse, B, H, N_q, N_k, d, scale, causal, l
     return int(load_library().fa_selftest_fwd_timeout(
         _addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(H), int(N_q), int(N_k),
         int(d), float(scale), int(bool(causal)), int(limit_cycles), _stream(stream)))
+
+
+def fa_selftest_bwd_timeout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, d, scale, causal,
+                            workspace, workspace_bytes, limit_cycles, stream=None) -> int:
+    """``fa_selftest_bwd_timeout`` of include/fa.h: the backward kernel with a short wait limit."""
+    return int(load_library().fa_selftest_bwd_timeout(
+        _addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(dout), _addr(dq), _addr(dk),
+        _addr(dv), int(B), int(H), int(N_q), int(N_k), int(d), float(scale), int(bool(causal)),
+        _addr(workspace), int(workspace_bytes), int(limit_cycles), _stream(stream)))
 
 
 def attention(q, k, v, causal=False, key_lens=None, scale=None, stream=None):

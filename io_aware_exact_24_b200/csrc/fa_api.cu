@@ -503,7 +503,8 @@ BwdLayout bwd_layout(int B, int H, int N_q, int d) {
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                void* dq, void* dk, void* dv, int B, int H, int N_q, int N_k, float scale, int causal,
-               const int32_t* key_lens, uint8_t* ws, cudaStream_t stream) {
+               const int32_t* key_lens, uint8_t* ws, cudaStream_t stream,
+               unsigned long long wait_limit = kWaitLimitCycles) {
     const BwdLayout L = bwd_layout(B, H, N_q, D);
     float* dsum = reinterpret_cast<float*>(ws + L.dsum);
     float* dq_acc = reinterpret_cast<float*>(ws + L.dq_acc);
@@ -545,7 +546,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         p.scale = scale;
         p.scale_log2 = scale * 1.4426950408889634f;
         p.causal = causal ? 1 : 0;
-        p.wait_limit = kWaitLimitCycles;
+        p.wait_limit = wait_limit;
         dim3 grid((unsigned)((N_k + 127) / 128), (unsigned)H, (unsigned)B);
         fa::fa_bwd_sm100_kernel<D><<<grid, fa::kBwdThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
         e = cudaGetLastError();
@@ -783,9 +784,12 @@ size_t fa_bwd_workspace_size(int B, int H, int N_q, int d) {
     return bwd_layout(B, H, N_q, d).total;
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
-           void* dk, void* dv, int B, int H, int N_q, int N_k, int d, float scale, int causal,
-           const int32_t* key_lens, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+// fa_bwd's argument checks and launch; wait_limit bounds every pipeline wait of the
+// main kernel (the default outside the self test).
+static int bwd_entry(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int H, int N_q, int N_k, int d, float scale, int causal,
+                     const int32_t* key_lens, void* workspace, size_t workspace_bytes, fa_stream_t stream,
+                     unsigned long long wait_limit) {
     bool empty = false;
     int st = validate(q, k, v, o, lse, B, H, N_q, N_k, d, scale, key_lens, &empty);
     if (st != FA_OK) return st;
@@ -813,8 +817,17 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (d == 64)
-        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s);
-    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s);
+        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s,
+                              wait_limit);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, scale, causal, key_lens, ws, s,
+                           wait_limit);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int H, int N_q, int N_k, int d, float scale, int causal,
+           const int32_t* key_lens, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, d, scale, causal, key_lens, workspace,
+                     workspace_bytes, stream, kWaitLimitCycles);
 }
 
 int fa_fwd_bias(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_q, int N_k,
@@ -1094,6 +1107,18 @@ int fa_selftest_fwd_timeout(const void* q, const void* k, const void* v, void* o
                                 limit_cycles)
                    : launch<128>(q, k, v, o, lse, B, H, N_q, N_k, scale, causal, nullptr, s, none, -1, nob, 1.f,
                                  limit_cycles);
+    if (st != FA_OK) return st;
+    return fa_get_device_status(stream);
+}
+
+int fa_selftest_bwd_timeout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, int B, int H, int N_q, int N_k, int d,
+                            float scale, int causal, void* workspace, size_t workspace_bytes,
+                            unsigned long long limit_cycles, fa_stream_t stream) {
+    if (limit_cycles < 1 || limit_cycles > (1ull << 32)) return FA_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N_q <= 0 || N_k <= 0) return FA_ERR_INVALID_ARG;   // nothing would wait
+    const int st = bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, B, H, N_q, N_k, d, scale, causal, nullptr,
+                             workspace, workspace_bytes, stream, limit_cycles);
     if (st != FA_OK) return st;
     return fa_get_device_status(stream);
 }

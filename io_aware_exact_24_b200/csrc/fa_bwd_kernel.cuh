@@ -114,15 +114,6 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                  : "memory");
 }
 
-// Waits for asynchronous work that completes on its own (copies already issued,
-// MMAs already issued) -- even after another role gave up -- so that nothing is
-// still writing shared memory or TMEM when the CTA releases them.  Bounded.
-__device__ __forceinline__ void wait_own_work(uint32_t bar, uint32_t parity, unsigned long long limit) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if ((unsigned long long)(clock64() - t0) > limit) break;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -239,14 +230,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 bx * 64, q0, h, b, pol_keep);
                 ++no;
             }
-            // wind down: every copy issued lands before the CTA exits
-            wait_own_work(bar_kv, 0, p.wait_limit);
-            if (!ok) {
-                for (int c2 = (nq > C::kStagesQ ? nq - C::kStagesQ : 0); c2 < nq; ++c2)
-                    wait_own_work(bar_q_full(c2 % C::kStagesQ), (uint32_t)((c2 / C::kStagesQ) & 1), p.wait_limit);
-                for (int c2 = (no > C::kStagesO ? no - C::kStagesO : 0); c2 < no; ++c2)
-                    wait_own_work(bar_o_full(c2 % C::kStagesO), (uint32_t)((c2 / C::kStagesO) & 1), p.wait_limit);
-            }
+            // wind down: every copy issued lands before the CTA exits, also when a
+            // consumer gave up after this producer issued its last copy (the waits
+            // ignore the abort flag and keep the default limit, whatever the
+            // caller's; on the normal path the phases are complete already).  Only
+            // the newest copy of each slot can still be in flight.
+            (void)wait_own_work(bar_kv, 0);
+            for (int c2 = (nq > C::kStagesQ ? nq - C::kStagesQ : 0); c2 < nq; ++c2)
+                (void)wait_own_work(bar_q_full(c2 % C::kStagesQ), (uint32_t)((c2 / C::kStagesQ) & 1));
+            for (int c2 = (no > C::kStagesO ? no - C::kStagesO : 0); c2 < no; ++c2)
+                (void)wait_own_work(bar_o_full(c2 % C::kStagesO), (uint32_t)((c2 / C::kStagesO) & 1));
         }
         __syncwarp();
     } else if (warp == kBwdMmaWarp) {
@@ -326,9 +319,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 umma_commit(bar_dq_full);
             }
-            // every MMA issued has completed before TMEM is released (also after a give-up)
+            // every MMA issued has completed before TMEM is released (also after a
+            // give-up; this wait ignores the abort flag and the caller's limit)
             umma_commit(bar_drain);
-            wait_own_work(bar_drain, 0, p.wait_limit);
+            (void)wait_own_work(bar_drain, 0);
         }
         __syncwarp();
     } else if (warp >= kBwdComputeWarp0) {

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("fa_fwd", "fa_fwd_host", "fa_fwd_host_workspace_size", "fa_status_string",
                  "fa_get_device_status", "fa_version", "fa_selftest_wait_timeout",
-                 "fa_selftest_fwd_timeout"):
+                 "fa_selftest_fwd_timeout", "fa_selftest_bwd_timeout"):
         assert must in names
 
 
@@ -284,6 +284,17 @@ def test_selftest_fwd_timeout_argument_errors(lib):
     assert f(limit=0) == binding.FA_ERR_INVALID_ARG
     assert f(limit=(1 << 32) + 1) == binding.FA_ERR_INVALID_ARG
     assert f(Nk=0) == binding.FA_ERR_INVALID_ARG
+    assert f(B=0) == binding.FA_ERR_INVALID_ARG
+
+
+def test_selftest_bwd_timeout_argument_errors(lib):
+    f = lambda **kw: binding.fa_selftest_bwd_timeout(
+        P, P, P, P, P, P, P, P, P, kw.get("B", 1), 2, kw.get("Nq", 8), kw.get("Nk", 8), 64, 0.125, 1,
+        P, 1 << 20, kw.get("limit", 2), stream=0)
+    assert f(limit=0) == binding.FA_ERR_INVALID_ARG
+    assert f(limit=(1 << 32) + 1) == binding.FA_ERR_INVALID_ARG
+    assert f(Nk=0) == binding.FA_ERR_INVALID_ARG
+    assert f(Nq=0) == binding.FA_ERR_INVALID_ARG
     assert f(B=0) == binding.FA_ERR_INVALID_ARG
 
 

@@ -64,3 +64,44 @@ def test_forward_wait_limit_runs_out_and_context_survives(d, causal, B, H, N):
     o_ref, lse_ref = oracle.attn_ref(q, k, v, scale, causal, None)
     compare(o2, lse2, o_ref, lse_ref, f"after forward timeout d={d}")
     assert fa_get_device_status() == FA_OK
+
+
+@pytest.mark.parametrize("d,causal,B,H,N", [(64, False, 1, 2, 700), (128, True, 1, 2, 700)],
+                         ids=["d64", "d128-causal"])
+def test_backward_wait_limit_runs_out_and_context_survives(d, causal, B, H, N):
+    # The backward kernel with a wait limit of a few cycles: some pipeline wait runs
+    # out, every role of that CTA stops after its own copies, MMAs and dQ reduce-adds
+    # have landed, and the call reports FA_ERR_DEVICE_TIMEOUT.  Afterwards a normal
+    # backward call passes its derived bound and leaves the status clean.  At d = 64
+    # the kernel also copies K and V into TMEM, whose barrier winds down the same way.
+    import torch
+    from io_aware_exact_24_b200 import (FA_ERR_DEVICE_TIMEOUT, FA_OK, fa_bwd_workspace_size, fa_fwd,
+                                        fa_get_device_status, fa_selftest_bwd_timeout)
+    from fa_testutil import to_device_bf16
+    from io_aware_exact_24_b200.inputs import TENSOR_DO
+    from test_gpu_bwd import bounds, run_fwd_bwd
+    assert fa_get_device_status() == FA_OK
+    q = normal_bf16((B, H, N, d), 40 + d, 0)
+    k = normal_bf16((B, H, N, d), 40 + d, 1)
+    v = normal_bf16((B, H, N, d), 40 + d, 2)
+    do = normal_bf16((B, H, N, d), 40 + d, TENSOR_DO)
+    scale = float(np.float32(1 / np.sqrt(d)))
+    tq, tk, tv, tdo = (to_device_bf16(x) for x in (q, k, v, do))
+    o = torch.empty_like(tq)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    fa_fwd(tq, tk, tv, o, lse, B, H, N, N, d, scale, causal, None)
+    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+    nbytes = fa_bwd_workspace_size(B, H, N, d)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        st = fa_selftest_bwd_timeout(tq, tk, tv, o, lse, tdo, dq, dk, dv, B, H, N, N, d, scale, causal,
+                                     ws, nbytes, 2)
+        assert st == FA_ERR_DEVICE_TIMEOUT
+        assert fa_get_device_status() == FA_OK      # read and cleared by the call
+    o2, lse2, gq, gk, gv = run_fwd_bwd(q, k, v, do, scale, causal, None)
+    rq, rk, rv, bq, bk, bv, o_ref, lse_ref = bounds(q, k, v, do, scale, causal, None, o2, lse2)
+    compare(o2, lse2, o_ref, lse_ref, f"forward after backward timeout d={d}")
+    for name, g, r, bd in (("dQ", gq, rq, bq), ("dK", gk, rk, bk), ("dV", gv, rv, bv)):
+        ratio = float((np.abs(g - r) / bd).max())
+        assert ratio <= 1.0, f"after backward timeout d={d}: {name} at x{ratio:.3f} of its bound"
+    assert fa_get_device_status() == FA_OK
