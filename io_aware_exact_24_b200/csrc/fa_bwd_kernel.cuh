@@ -17,18 +17,22 @@
 //  * warp 0 (one lane): TMA loads of K_j and V_j once, then Q_i and dO_i per
 //    query tile (Q and dO in rings of their own: kStagesQ / kStagesO slots);
 //  * warp 1 (one lane): the five tcgen05 MMAs of a tile --
-//      S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T     (M = 128 keys, N = 128 queries)
-//      dV  += P^T dO_i    and  dK  += dS^T Q_i       (A = P^T / dS^T from TMEM)
+//      S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T     (M = 128 keys, N = 128 queries;
+//                                                      at d = 64 A = K_j / V_j from TMEM)
+//      dV  += P^T dO_i    and  dK  += dS^T Q_i       (A = P^T / dS^T from TMEM, issued
+//                                                      per compute pass)
 //      dQ_i = dS K_j                                  (A = dS^T from shared memory,
 //                                                      MN-major: M = queries)
 //    dV and dK stay in TMEM for the whole CTA;
-//  * warps 4-11, two per TMEM lane quadrant, each thread one key row and half
-//    of the columns: P^T and dS^T from S^T and dP^T (exp2 domain, masks),
-//    written back to TMEM as bf16 over the columns just read and, for dS^T, to
-//    shared memory; then each thread reads half of one query row of dQ_i and
-//    adds it into the fp32 dQ accumulator in global memory (vector atomic adds:
-//    several key blocks update each query row); finally dV and scale * dK go to
-//    global memory as bf16.
+//  * warps 4-11, two per TMEM lane quadrant, each thread one key row: in two
+//    passes of 32 queries each, P^T and dS^T from S^T and dP^T (exp2 domain,
+//    masks), written back to TMEM as bf16 over the columns just read and, for
+//    dS^T, to shared memory, each pass handed to the issuer on its own barrier;
+//    then each thread reads half of one query row of dQ_i, stages it in shared
+//    memory and adds it into the fp32 dQ accumulator in global memory with a TMA
+//    tensor reduce-add (several key blocks update each query row); finally dV
+//    and scale * dK go to global memory as bf16.  At d = 64 they first copy the
+//    block's K and V rows into TMEM.
 // Every mbarrier wait is bounded (as in the forward kernel); a wait that runs
 // out records FA_ERR_DEVICE_TIMEOUT and the CTA winds down.
 #pragma once
@@ -108,11 +112,6 @@ struct BwdCfg {
     static constexpr uint32_t kIdescQ = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                         (((uint32_t)D >> 3) << 17) | ((128u >> 4) << 24);
 };
-
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
