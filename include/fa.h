@@ -279,9 +279,11 @@ FA_API size_t fa_fwd_host_workspace_size(int B, int H, int N_q, int N_k, int d,
  *
  * Copies the inputs to the workspace, runs fa_fwd on `stream`, copies O and
  * LSE back, and synchronises `stream` before returning, so on FA_OK the host
- * outputs are complete.  The work is cut into chunks of about 1/16 of the
+ * outputs are complete.  The work is cut into chunks of about 1/8 of the
  * (batch, head) pairs (runs of heads of one batch entry, or whole batch
- * entries), each its own fa_fwd launch; the library's own copy streams move
+ * entries; with runs of heads the last chunk is cut further into halves, so
+ * little work is left after the last input copy), each its own fa_fwd
+ * launch; the library's own copy streams move
  * chunk c+1 in and chunk c-1 out while chunk c runs (it waits for earlier work
  * on `stream` before touching the workspace).  The result is the same, bit for
  * bit, as fa_fwd on the whole problem.  Calls on one device are serialised.  Returns FA_ERR_INVALID_ARG if the workspace is too

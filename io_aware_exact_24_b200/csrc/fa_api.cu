@@ -55,7 +55,7 @@ constexpr int kPersistMaxTiles = 16;
 constexpr int kMaxDevices = 64;
 // fa_fwd_host pipelines its copies in chunks of heads: about this many chunks,
 // at most kHostChunksMax
-constexpr int kHostChunksTarget = 16;
+constexpr int kHostChunksTarget = 8;
 constexpr int kHostChunksMax = 64;
 // largest relative-position radius of a bias table (2^30: the table's
 // 2R+1 entries and every clamped index stay within int range)
@@ -984,11 +984,41 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse
     const long long want = (total + kHostChunksTarget - 1) / kHostChunksTarget;   // pairs per chunk
     const bool by_heads = want <= H;
     const int per = by_heads ? (int)std::max(1LL, want) : H;                      // heads per chunk
-    const int per_b = by_heads ? (H + per - 1) / per : 1;                         // chunks per batch entry
     const int bc = by_heads ? 1 : (int)((want + H - 1) / H);                      // batch entries per chunk
-    const int n_chunks = by_heads ? B * per_b : (B + bc - 1) / bc;
-    // at most 2 * kHostChunksTarget chunks (heads: B <= target; batches: <= target)
-    if (n_chunks > kHostChunksMax) return FA_ERR_UNSUPPORTED;
+    // Chunks as (first batch entry, batch entries, first head, heads).  What is left
+    // after the last host-to-device copy -- the last chunk's forward and read-back --
+    // is not overlapped, so with chunks of heads the last chunk is cut into halves
+    // (per/2, per/4, .., 1, 1 heads): the tail is about one head's work.
+    struct Chunk { int b, nb, h0, hc; };
+    Chunk chunks[kHostChunksMax];
+    int n_chunks = 0;
+    if (by_heads) {
+        for (int b = 0; b < B; ++b)
+            for (int h0 = 0; h0 < H; h0 += per) {
+                const int hc = std::min(per, H - h0);
+                if (b == B - 1 && h0 + hc == H) {
+                    int left = hc, at = h0;
+                    while (left > 1 && n_chunks < kHostChunksMax) {
+                        const int half = left / 2;
+                        chunks[n_chunks++] = {b, 1, at, left - half};
+                        at += left - half;
+                        left = half;
+                    }
+                    if (left > 0) {
+                        if (n_chunks >= kHostChunksMax) return FA_ERR_UNSUPPORTED;
+                        chunks[n_chunks++] = {b, 1, at, left};
+                    }
+                } else {
+                    if (n_chunks >= kHostChunksMax) return FA_ERR_UNSUPPORTED;
+                    chunks[n_chunks++] = {b, 1, h0, hc};
+                }
+            }
+    } else {
+        for (int b = 0; b < B; b += bc) {
+            if (n_chunks >= kHostChunksMax) return FA_ERR_UNSUPPORTED;
+            chunks[n_chunks++] = {b, std::min(bc, B - b), 0, H};
+        }
+    }
     // the workspace may still be in use by earlier work on `stream`
     e = cudaEventRecord(hp->start, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
@@ -1000,10 +1030,8 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse
     }
     if (e != cudaSuccess) return cuda_fail("fa_fwd_host setup", e);
     for (int c = 0; c < n_chunks; ++c) {
-        const int b = by_heads ? c / per_b : c * bc;
-        const int nb = by_heads ? 1 : std::min(bc, B - b);     // batch entries of the chunk
-        const int h0 = by_heads ? (c % per_b) * per : 0;
-        const int hc = by_heads ? std::min(per, H - h0) : H;   // heads per batch entry
+        const int b = chunks[c].b, nb = chunks[c].nb;           // batch entries of the chunk
+        const int h0 = chunks[c].h0, hc = chunks[c].hc;         // heads per batch entry
         const size_t row0 = (size_t)b * H + h0;                 // first (b, h) pair of the chunk
         const size_t rows = (size_t)nb * hc;                    // (b, h) pairs of the chunk
         e = cudaMemcpyAsync(ws + L.q + row0 * q_head, static_cast<const char*>(q) + row0 * q_head, rows * q_head,
