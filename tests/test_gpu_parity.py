@@ -180,12 +180,14 @@ def test_zero_query_gives_mean_of_values():
 
 
 @pytest.mark.parametrize("shape", [(2, 3, 333, 257, 128, True), (2, 20, 300, 300, 64, False),
-                                   (40, 2, 200, 150, 64, True)],
-                         ids=["heads-6-chunks", "heads-20-per-batch", "whole-batches"])
+                                   (1, 64, 130, 200, 64, True), (40, 2, 200, 150, 64, True)],
+                         ids=["heads-6-chunks", "heads-5-per-chunk-tail-3-1-1", "heads-8-per-chunk-tail-4-2-1-1",
+                              "whole-batches"])
 def test_host_entry_matches_device_entry(shape):
     # the host entry copies and computes in chunks of heads (or of whole batch
-    # entries when a batch entry is small); every chunk is its own launch, and the
-    # result must be the device entry's, bit for bit
+    # entries when a batch entry is small), the last chunk of heads cut into
+    # halves; every chunk is its own launch, and the result must be the device
+    # entry's, bit for bit
     import torch
     from io_aware_exact_24_b200 import fa_fwd_host, fa_fwd_host_workspace_size
     B, H, Nq, Nk, d, with_kl = shape
