@@ -304,7 +304,7 @@ def fp8_table(steps, warmup, device, peak_bf16_tflops):
 
 
 def time_bwd(w, x, steps, warmup, device):
-    """Mean per-call device time (ms) of fa_bwd (its four launches) on resident inputs,
+    """Mean per-call device time (ms) of fa_bwd (its three kernels) on resident inputs,
     the forward's O and LSE computed once beforehand; L2 flushed between calls."""
     import torch
     from io_aware_exact_24_b200 import fa_bwd, fa_bwd_workspace_size, fa_fwd

@@ -211,14 +211,15 @@ FA_API int fa_fwd_fp8(const void *q8, const void *k8, const void *v8, void *o, f
  *   workspace     device, 256-byte aligned, at least fa_bwd_workspace_size(B,H,N_q,d)
  *                 bytes, owned by the caller; overwritten (D and an fp32 dQ
  *                 accumulator). Calls sharing a workspace must be ordered.
- *   stream        as for fa_fwd; four launches are enqueued (D and zeroing, the
- *                 main kernel, dQ to bf16).
+ *   stream        as for fa_fwd; three kernels are enqueued (D and zeroing, the
+ *                 main kernel, dQ to bf16; with N_q = 0 two memsets instead).
  *
  * Returns FA_OK once enqueued.  Errors as fa_fwd, plus FA_ERR_INVALID_ARG for a
  * NULL or short workspace or NULL gradient buffers, FA_ERR_MISALIGNED for
  * unaligned dout/dq/dk/dv/workspace.  B = 0 or H = 0: no-op.  N_q = 0: dk = dv = 0.
- * N_k = 0: dq = 0.  The dQ sums use atomic adds, so dq may differ in the last
- * bits between runs; dk and dv are deterministic.
+ * N_k = 0: dq = 0.  The dQ sums across key blocks are tensor reduce-adds (atomic
+ * at L2, in arrival order), so dq may differ in the last bits between runs; dk
+ * and dv are deterministic.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N_q, int d);
 FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
